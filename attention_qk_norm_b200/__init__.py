@@ -1,1 +1,18 @@
-"""QK-Norm for B200 (placeholder until the CUDA library lands)."""
+"""QK-Norm on NVIDIA B200: per-head and layerwise (SwiftQK) RMSNorm of Q/K.
+
+The compute lives in ``libqknorm.so`` (hand-written CUDA for sm_100a, C ABI
+in ``include/qknorm.h``).  This package holds its build script, a thin
+ctypes binding with the same entry-point names, and ``synth`` (seeded
+synthetic inputs).  The library is loaded on first use, so importing the
+package, or ``synth`` alone, needs neither the library nor a GPU.
+"""
+from ._binding import (  # noqa: F401
+    QKN_BF16,
+    QKN_FP32,
+    QKNormError,
+    load_library,
+    qknorm_layerwise,
+    qknorm_per_head,
+    status_string,
+)
+from .buildlib import LIB_PATH, build  # noqa: F401

@@ -1,0 +1,139 @@
+"""ctypes binding of libqknorm.so: argument marshalling only.
+
+Every step of QK-Norm runs in the library's CUDA kernels; this module turns
+torch tensors into pointers, sizes and a stream handle, calls the C entry
+point of the same name, and raises ``QKNormError`` on a non-zero status.
+There is no fallback: if the library is missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from .buildlib import LIB_PATH
+
+QKN_BF16, QKN_FP32 = 0, 1
+STATUS = {
+    0: "QKN_OK", -1: "QKN_ERR_NULL", -2: "QKN_ERR_SHAPE", -3: "QKN_ERR_ALIGN",
+    -4: "QKN_ERR_NSHARDS", -5: "QKN_ERR_UNSUPPORTED", -6: "QKN_ERR_CUDA", -7: "QKN_ERR_EPS",
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class QKNormError(RuntimeError):
+    """A non-zero qkn_status returned by libqknorm.so."""
+
+    def __init__(self, fn: str, status: int, message: str, cuda_error: int = 0):
+        self.status = status
+        self.cuda_error = cuda_error
+        extra = " (cudaError %d)" % cuda_error if status == -6 else ""
+        super().__init__("%s: %s [%s]%s" % (fn, message, STATUS.get(status, status), extra))
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libqknorm.so and declare its prototypes (include/qknorm.h)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path == LIB_PATH:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                "libqknorm.so is not built at %s; run `python -m attention_qk_norm_b200.buildlib` "
+                "(QK-Norm has no non-CUDA path)" % path)
+        lib = ctypes.CDLL(path)
+        vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        lib.qknorm_per_head.argtypes = [vp, i32, i64, i32, i32, i32, i64, vp, vp, f32, vp]
+        lib.qknorm_per_head.restype = i32
+        lib.qknorm_layerwise.argtypes = [vp, i32, i64, i32, i32, i32, i64, vp, vp, f32, i32, vp]
+        lib.qknorm_layerwise.restype = i32
+        lib.qknorm_status_string.argtypes = [i32]
+        lib.qknorm_status_string.restype = ctypes.c_char_p
+        lib.qknorm_last_cuda_error.argtypes = []
+        lib.qknorm_last_cuda_error.restype = i32
+        lib.qknorm_version.argtypes = []
+        lib.qknorm_version.restype = i32
+        if path == LIB_PATH:
+            _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().qknorm_status_string(int(status)).decode()
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        lib = load_library()
+        raise QKNormError(fn, rc, lib.qknorm_status_string(rc).decode(),
+                          lib.qknorm_last_cuda_error())
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return QKN_BF16
+    if t.dtype == torch.float32:
+        return QKN_FP32
+    raise TypeError("qkv must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _rows(qkv, row_stride):
+    if qkv.dim() != 2 or qkv.stride(1) != 1:
+        raise ValueError("qkv must be a 2-D [T, row_stride] view with unit column stride")
+    stride = qkv.stride(0) if row_stride is None else int(row_stride)
+    return qkv.shape[0], stride
+
+
+def _stream_ptr(qkv, stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(qkv.device)
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _gamma_ptr(g, name):
+    import torch
+
+    if g is None:
+        return None
+    if g.dtype != torch.float32 or not g.is_contiguous():
+        raise TypeError("%s must be a contiguous float32 tensor" % name)
+    return ctypes.c_void_p(g.data_ptr())
+
+
+def _device_check(qkv, *gammas):
+    if not qkv.is_cuda:
+        raise ValueError("qkv must be a CUDA tensor (QK-Norm runs only on the GPU)")
+    for g in gammas:
+        if g is not None and g.device != qkv.device:
+            raise ValueError("gamma must live on the same device as qkv")
+
+
+def qknorm_per_head(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, row_stride=None, stream=None):
+    """Per-head QK-Norm in place on ``qkv`` [T, row_stride] (see qknorm.h)."""
+    _device_check(qkv, gamma_q, gamma_k)
+    T, stride = _rows(qkv, row_stride)
+    rc = load_library().qknorm_per_head(
+        ctypes.c_void_p(qkv.data_ptr()), _dtype_code(qkv), T, Hq, Hk, D, stride,
+        _gamma_ptr(gamma_q, "gamma_q"), _gamma_ptr(gamma_k, "gamma_k"), float(eps),
+        _stream_ptr(qkv, stream))
+    _check("qknorm_per_head", rc)
+    return qkv
+
+
+def qknorm_layerwise(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, nshards=1, row_stride=None,
+                     stream=None):
+    """Layerwise (SwiftQK) QK-Norm in place on ``qkv`` [T, row_stride]."""
+    _device_check(qkv, gamma_q, gamma_k)
+    T, stride = _rows(qkv, row_stride)
+    rc = load_library().qknorm_layerwise(
+        ctypes.c_void_p(qkv.data_ptr()), _dtype_code(qkv), T, Hq, Hk, D, stride,
+        _gamma_ptr(gamma_q, "gamma_q"), _gamma_ptr(gamma_k, "gamma_k"), float(eps),
+        int(nshards), _stream_ptr(qkv, stream))
+    _check("qknorm_layerwise", rc)
+    return qkv

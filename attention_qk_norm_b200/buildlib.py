@@ -1,0 +1,53 @@
+"""Build ``libqknorm.so`` in-tree with nvcc for sm_100a.
+
+The library links the CUDA runtime statically, so it loads on a host
+without a GPU (argument validation needs no device) and does not depend on
+the runtime version torch ships.
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+INCLUDE = os.path.join(ROOT, "include")
+SOURCES = [os.path.join(PKG, "csrc", "qknorm.cu")]
+HEADERS = [os.path.join(INCLUDE, "qknorm.h")]
+LIB_PATH = os.path.join(PKG, "libqknorm.so")
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-lineinfo", "-O3", "-std=c++17",
+    "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
+]
+
+
+def nvcc() -> str:
+    found = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(found):
+        raise RuntimeError("nvcc not found; the CUDA toolkit is required to build libqknorm.so")
+    return found
+
+
+def is_stale() -> bool:
+    if not os.path.exists(LIB_PATH):
+        return True
+    t = os.path.getmtime(LIB_PATH)
+    return any(os.path.getmtime(p) > t for p in SOURCES + HEADERS)
+
+
+def build(force: bool = False, extra_flags=(), out: str = LIB_PATH) -> str:
+    """Compile the CUDA sources into ``out`` when stale (or always if forced)."""
+    if not force and out == LIB_PATH and not is_stale():
+        return out
+    tmp = out + ".%d.tmp" % os.getpid()
+    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, *SOURCES, "-o", tmp]
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(force=True))

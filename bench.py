@@ -1,0 +1,551 @@
+#!/usr/bin/env python
+"""Benchmark of QK-Norm on B200: tokens/s and achieved HBM GB/s against T.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one call of the hot path over one batch: per-head QK-Norm of the
+head_dim-128, 48-head, T=4096 bf16 workload (the shape of the sglang /
+turbomind kernel table's largest row), in place, through the C ABI.  Steps
+rotate over enough copies of the input that the set is more than four times
+the L2 cache, so every step reads from HBM.  Launches are replayed from CUDA
+graphs of up to 100 steps; the timed region is exactly K steps between a
+barrier plus device synchronisation on both sides, timed with CUDA events
+on the launching stream, max over ranks.
+
+Rank 0 prints one JSON line.  Besides the headline it carries the roofline
+of the kernel, an end-to-end figure through host buffers, the CPU oracle as
+a reported baseline, SM clocks sampled during the timed region, and a sweep
+over T and over the other workloads (GQA fused layout, layerwise with 1..8
+emulated shards, fp32 / head_dim 64..256 stress shapes).
+
+Under torchrun with N > 1 every rank runs the same per-GPU workload on its
+own GPU (weak scaling: tokens are independent, so no collective touches the
+data; NCCL carries only the barrier and the max of the timings).
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead
+(rank 0 only), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "QK-Norm tokens/s and achieved HBM GB/s (fraction of B200 peak) vs T"
+UNIT = "tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+GRAPH_STEPS = 100
+
+HEADLINE = dict(kind="per_head", T=4096, Hq=48, Hk=0, D=128, dtype="bf16", eps=1e-6, nshards=1,
+                seed=1001)
+HEADLINE_NAME = ("per-head QK-Norm, head_dim 128, 48 heads, T=4096 tokens, bf16, Q-style "
+                 "contiguous [T,48,128] (shape of the largest row of the sglang/turbomind "
+                 "kernel table)")
+
+
+# ---------------------------------------------------------------- helpers --
+def workload_bytes(w) -> int:
+    """Algorithmic bytes of one call: read + write of Q and K once, gamma once."""
+    es = 2 if w["dtype"] == "bf16" else 4
+    qk = (w["Hq"] + w["Hk"]) * w["D"]
+    if w["kind"] == "per_head":
+        gamma = w["D"] * 4 * ((w["Hq"] > 0) + (w["Hk"] > 0))
+    else:
+        gamma = qk * 4
+    return 2 * w["T"] * qk * es + gamma
+
+
+def row_stride(w) -> int:
+    return (w["Hq"] + 2 * w["Hk"]) * w["D"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record():
+    """Committed ncu DRAM bytes per launch, valid only for the kernel source
+    they were taken from (hash of csrc/qknorm.cu)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "attention_qk_norm_b200", "csrc", "qknorm.cu")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        return rec if rec.get("source_sha256") == sha else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        with open(self.out.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.out.name)
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------- distributed --
+def dist_init():
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local) if backend == "nccl" else None)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def shard_units(total: int, world: int, rank: int):
+    """Contiguous split of ``total`` independent units over ranks (for runs
+    that divide one fixed job; the benchmark itself runs weak scaling)."""
+    base, rem = divmod(total, world)
+    start = rank * base + min(rank, rem)
+    return start, start + base + (1 if rank < rem else 0)
+
+
+# ---------------------------------------------------------------- GPU side --
+class Workload:
+    """Device buffers of one workload, rotated so their total exceeds 4x L2."""
+
+    def __init__(self, w, device, l2_bytes, max_bytes=16 << 30):
+        import torch
+        from attention_qk_norm_b200 import synth
+
+        self.w = w
+        d = synth.make_case_torch(w["T"], w["Hq"], w["Hk"], w["D"], device=device,
+                                  dtype=w["dtype"], seed=w["seed"], eps=w["eps"],
+                                  layerwise=w["kind"] == "layerwise",
+                                  scale=w.get("scale"), zero_frac=w.get("zero_frac", 0.0),
+                                  outlier_frac=w.get("outlier_frac", 0.0))
+        self.gq, self.gk = d["gamma_q"], d["gamma_k"]
+        one = d["qkv"].numel() * d["qkv"].element_size()
+        n = max(2, math.ceil(4 * l2_bytes / max(1, one)))
+        n = max(1, min(n, max_bytes // max(1, one)))
+        self.bufs = [d["qkv"]] + [d["qkv"].clone() for _ in range(n - 1)]
+        self.buffer_bytes = one
+        self.host_in = None
+        self.i = 0
+        torch.cuda.synchronize()
+
+    def launch(self, buf=None):
+        import attention_qk_norm_b200 as qkn
+
+        w = self.w
+        if buf is None:
+            buf = self.bufs[self.i % len(self.bufs)]
+            self.i += 1
+        if w["kind"] == "per_head":
+            qkn.qknorm_per_head(buf, w["Hq"], w["Hk"], w["D"], self.gq, self.gk, w["eps"])
+        else:
+            qkn.qknorm_layerwise(buf, w["Hq"], w["Hk"], w["D"], self.gq, self.gk, w["eps"],
+                                 nshards=w["nshards"])
+
+    def graph(self, steps: int):
+        import torch
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(steps):
+                self.launch()
+        return g
+
+    def free(self):
+        self.bufs = []
+
+
+def time_graph_us(wl, reps=5, min_ms=20.0):
+    """Median per-launch time (µs) over `reps` timed groups of graph replays."""
+    import torch
+
+    g = wl.graph(GRAPH_STEPS)
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    g.replay()
+    e.record()
+    e.synchronize()
+    per = max(s.elapsed_time(e), 1e-3)
+    n = max(1, int(math.ceil(min_ms / per)))
+    samples = []
+    for _ in range(reps):
+        s.record()
+        for _ in range(n):
+            g.replay()
+        e.record()
+        e.synchronize()
+        samples.append(s.elapsed_time(e) * 1e3 / (n * GRAPH_STEPS))
+    del g
+    return statistics.median(samples)
+
+
+def point(w, us, hbm_peak):
+    b = workload_bytes(w)
+    gbs = b / (us * 1e-6) / 1e9
+    return {"T": w["T"], "us": round(us, 3), "tokens_per_s": round(w["T"] / (us * 1e-6), 1),
+            "gbs": round(gbs, 1), "frac_measured": round(gbs / hbm_peak, 4),
+            "frac_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "bytes": b}
+
+
+def extra_workloads():
+    from attention_qk_norm_b200 import synth
+
+    out = []
+    for T in synth.SWEEP_T:
+        out.append(("sweep H=48", dict(HEADLINE, T=T, seed=2000 + T)))
+    for H in (16, 32):
+        out.append(("sweep H=%d" % H, dict(HEADLINE, Hq=H, T=4096, seed=2100 + H)))
+    for T in synth.GQA_T:
+        out.append(("gqa fused 32q/8kv", dict(kind="per_head", T=T, Hq=32, Hk=8, D=128,
+                                              dtype="bf16", eps=1e-6, nshards=1,
+                                              scale="lognormal", seed=2200 + T)))
+    for n in synth.LAYERWISE_NSHARDS:
+        for T in synth.LAYERWISE_T:
+            out.append(("layerwise n=%d" % n, dict(kind="layerwise", T=T, Hq=32, Hk=8, D=128,
+                                                    dtype="bf16", eps=1e-6, nshards=n,
+                                                    seed=2300 + T)))
+    for dt in synth.STRESS_DTYPES:
+        for D in synth.STRESS_D:
+            for kind in ("per_head", "layerwise"):
+                out.append(("stress %s %s D=%d" % (kind, dt, D),
+                            dict(kind=kind, T=32768, Hq=64, Hk=8, D=D, dtype=dt, eps=1e-6,
+                                 nshards=8 if kind == "layerwise" else 1, scale="stress",
+                                 zero_frac=0.01, outlier_frac=0.01, seed=2400 + D)))
+    return out
+
+
+def run_extras(device, l2, hbm_peak):
+    import torch
+
+    res = []
+    for name, w in extra_workloads():
+        wl = Workload(w, device, l2, max_bytes=8 << 30)
+        for _ in range(3):
+            wl.launch()
+        us = time_graph_us(wl)
+        p = point(w, us, hbm_peak)
+        p["workload"] = name
+        res.append(p)
+        wl.free()
+        del wl
+        torch.cuda.empty_cache()
+    return res
+
+
+def e2e(w, device, steps):
+    """Same metric through host buffers: per step a pinned-host -> device copy
+    of the input, the C-ABI call, and a device -> pinned-host copy of the
+    normalised buffer, all inside the timed region."""
+    import torch
+    from attention_qk_norm_b200 import synth
+
+    d = synth.make_case_torch(w["T"], w["Hq"], w["Hk"], w["D"], device="cpu", dtype=w["dtype"],
+                              seed=w["seed"], eps=w["eps"])
+    host_in = d["qkv"].pin_memory()
+    host_out = torch.empty_like(host_in).pin_memory()
+    dev = torch.empty_like(host_in, device=device)
+    gq = d["gamma_q"].to(device)
+    wl = Workload.__new__(Workload)
+    wl.w, wl.gq, wl.gk = w, gq, None
+
+    def step():
+        dev.copy_(host_in, non_blocking=True)
+        wl.launch(dev)
+        host_out.copy_(dev, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    e.synchronize()
+    ms = s.elapsed_time(e)
+    nbytes = host_in.numel() * host_in.element_size()
+    return ms, nbytes
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The float64 oracle on the host cores, over whole copies of the
+    workload's input, for about `budget_s` seconds (at least one pass)."""
+    import oracle
+    from attention_qk_norm_b200 import synth
+
+    c = synth.make_case(w["T"], w["Hq"], w["Hk"], w["D"], dtype=w["dtype"], seed=w["seed"],
+                        eps=w["eps"])
+    threads = oracle.max_threads()
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        oracle.per_head(c.qkv, c.dtype, c.T, c.Hq, c.Hk, c.D, c.row_stride, c.gamma_q,
+                        c.gamma_k, c.eps, nthreads=threads)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (passes >= 1 and el * (passes + 1) / passes > 3 * budget_s):
+            break
+    return {"value": round(passes * c.T / el, 1), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": "%d full pass(es) of the %d-token workload (%.1f s)" % (passes, c.T, el)}
+
+
+# -------------------------------------------------------------- main arms --
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_init()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    props = torch.cuda.get_device_properties(device)
+    l2 = int(getattr(props, "L2_cache_size", 126 << 20))
+    hbm_peak, peak_kind = peaks()
+    w = dict(HEADLINE)
+    wl = Workload(w, device, l2)
+
+    for _ in range(args.warmup):
+        wl.launch()
+    torch.cuda.synchronize()
+    full, rem = divmod(args.steps, GRAPH_STEPS)
+    g_full = wl.graph(GRAPH_STEPS) if full else None
+    g_rem = wl.graph(rem) if rem else None
+    if g_full is not None:
+        g_full.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                           if world == 1 else local)
+    if rank == 0:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(full):
+        g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if rank == 0 else None
+    ms_local = s.elapsed_time(e)
+    ms = max_over_ranks(ms_local, world)
+    del g_full, g_rem
+
+    steps = args.steps
+    tokens = w["T"] * steps * world
+    value = tokens / (ms * 1e-3)
+    per_launch_us = ms_local * 1e3 / steps
+    b = workload_bytes(w)
+    achieved = b / (per_launch_us * 1e-6) / 1e9
+    tr = traffic_record()
+
+    e2e_ms, e2e_bytes = e2e(w, device, args.e2e_steps)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_val = w["T"] * args.e2e_steps * world / (e2e_ms * 1e-3)
+
+    l2_note = ("rotating %d in-place buffers of %.1f MB (%.0f MB > 4x L2 %.0f MB)"
+               % (len(wl.bufs), wl.buffer_bytes / 1e6, wl.buffer_bytes * len(wl.bufs) / 1e6,
+                  l2 / 1e6))
+    extras = None
+    if not args.no_extras:
+        wl.free()
+        torch.cuda.empty_cache()
+        extras = run_extras(device, l2, hbm_peak)
+    barrier(world)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms / steps, 6),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": HEADLINE_NAME, "T": w["T"], "heads": w["Hq"],
+                       "head_dim": w["D"], "kernel": "qknorm_per_head",
+                       "l2": l2_note,
+                       "launch": "CUDA graphs of %d launches" % GRAPH_STEPS,
+                       "parallelism": "dp%d (tokens independent, no collective)" % world},
+            "gpu_launches": steps,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1),
+                         "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(achieved / hbm_peak, 4),
+                         "peak_kind": peak_kind,
+                         "frac_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "algorithmic_bytes_per_launch": b,
+                         "traffic": tr["dram_bytes_per_launch"] if tr else None},
+            "e2e": {"value": round(e2e_val, 1), "unit": UNIT,
+                    "h2d_bytes_per_step": e2e_bytes, "d2h_bytes_per_step": e2e_bytes,
+                    "steps": args.e2e_steps},
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
+        if extras is not None:
+            line["sweep"] = extras
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The float64 CPU oracle on the workload's tokens, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    from attention_qk_norm_b200 import synth
+
+    w = HEADLINE
+    c = synth.make_case(w["T"], w["Hq"], w["Hk"], w["D"], dtype=w["dtype"], seed=w["seed"],
+                        eps=w["eps"])
+    threads = oracle.max_threads()
+
+    def step(n_tok, start):
+        rows = [(start + i) % c.T for i in range(n_tok)]
+        x = c.qkv[rows]
+        oracle.per_head(x, c.dtype, n_tok, c.Hq, c.Hk, c.D, c.row_stride, c.gamma_q, c.gamma_k,
+                        c.eps, nthreads=threads)
+
+    t0 = time.perf_counter()
+    step(256, 0)
+    per_tok = (time.perf_counter() - t0) / 256
+    budget = 120.0  # seconds for warm-up plus timed steps
+    n_tok = int(max(1, min(c.T, budget / max(1, args.steps + args.warmup) / max(per_tok, 1e-9))))
+    for i in range(args.warmup):
+        step(n_tok, i * n_tok)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(n_tok, (args.warmup + i) * n_tok)
+    el = time.perf_counter() - t0
+    value = args.steps * n_tok / el
+    sample = ("%d of the %d tokens per step (float64 oracle, %d threads)"
+              % (n_tok, c.T, threads))
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": HEADLINE_NAME, "T": w["T"], "heads": w["Hq"],
+                       "head_dim": w["D"]},
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-extras", action="store_true", help="skip the T / workload sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.steps < 1:
+        ap.error("--steps must be >= 1")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,122 @@
+/*
+ * qknorm.h -- C ABI of libqknorm.so: QK-Norm (RMSNorm of query and key
+ * activations) in place on a fused QKV activation buffer, on NVIDIA B200
+ * (sm_100a).
+ *
+ * Buffer layout ("combined QKV projection" lesson, GQA section: one fused
+ * projection output split by head into Q, K and V widths).  The activation
+ * is a row-major [T, row_stride] array of bf16 or fp32 in device memory:
+ *
+ *     columns [0, Hq*D)              Q   (Hq heads of head_dim D)
+ *     columns [Hq*D, (Hq+Hk)*D)      K   (Hk heads)
+ *     columns [(Hq+Hk)*D, W)         V   (Hk heads), W = (Hq + 2*Hk) * D
+ *     columns [W, row_stride)        padding
+ *
+ * Both entry points overwrite the Q and K columns of every row with their
+ * normalised values and never read or write V or the padding.
+ *
+ * Arithmetic: elements are widened to fp32, sums of squares accumulate in
+ * fp32, the inverse RMS is 1/sqrt(S/L + eps) in fp32 (L = normalised length,
+ * eps inside the square root), and each output x * rinv * gamma is rounded
+ * once to the storage type (round to nearest even for bf16).
+ *
+ * Common arguments
+ *   qkv         device pointer to the fused buffer; 16-byte aligned.
+ *   dtype       QKN_BF16 or QKN_FP32 (storage type of qkv).
+ *   T           number of tokens (rows), >= 0; T == 0 returns QKN_OK and
+ *               launches nothing (qkv may then be NULL).
+ *   Hq, Hk      query / key head counts, >= 0, Hq + Hk >= 1.
+ *   D           head_dim: 64, 128 or 256.
+ *   row_stride  elements between consecutive rows, >= W; row_stride *
+ *               sizeof(element) must be a multiple of 16 bytes.
+ *   gamma_q/k   fp32 device pointers, 16-byte aligned; gamma_k may be NULL
+ *               when Hk == 0 and gamma_q may be NULL when Hq == 0.
+ *   eps         finite, >= 0.
+ *   stream      a cudaStream_t passed as void* (NULL = legacy default stream).
+ *
+ * Ownership and execution: every pointer is owned by the caller and must
+ * stay valid until the work on `stream` completes.  The library allocates
+ * no memory and keeps no per-call state; calls are asynchronous and
+ * stream-ordered, and the caller synchronises.  Entry points are safe to call
+ * from several host threads.
+ *
+ * Errors: each entry point returns QKN_OK or a negative qkn_status and
+ * launches nothing when an argument is rejected.  Validation touches no CUDA
+ * API, so it runs on a host without a GPU.  QKN_ERR_CUDA means a CUDA runtime
+ * call (device query or kernel launch) failed on this call;
+ * qknorm_last_cuda_error() then returns that cudaError_t for the calling
+ * thread.
+ */
+#ifndef QKNORM_H
+#define QKNORM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { QKN_BF16 = 0, QKN_FP32 = 1 } qkn_dtype;
+
+typedef enum {
+    QKN_OK = 0,
+    QKN_ERR_NULL = -1,        /* a required pointer is NULL                     */
+    QKN_ERR_SHAPE = -2,       /* negative sizes, no heads, row_stride < W       */
+    QKN_ERR_ALIGN = -3,       /* qkv, gamma or row_stride bytes not 16-aligned  */
+    QKN_ERR_NSHARDS = -4,     /* nshards not in {1,2,4,8} or not dividing heads */
+    QKN_ERR_UNSUPPORTED = -5, /* dtype or head_dim not built, row too wide      */
+    QKN_ERR_CUDA = -6,        /* CUDA runtime error on this call                */
+    QKN_ERR_EPS = -7          /* eps negative or not finite                     */
+} qkn_status;
+
+/*
+ * Per-head QK-Norm (Qwen3 style).  Source: sglang PR #13189 "Add
+ * turbomind_rms_norm to accelerate QK norm in Qwen3 models", Motivation and
+ * Modifications (an RMSNorm whose hidden_size is head_dim), with the RMSNorm
+ * definition of the SwiftQK review (pith.science verdict for arXiv
+ * 2608.09160, core_discovery).  For every token t and head h < Hq + Hk, the
+ * D-element row x at columns [h*D, (h+1)*D) becomes
+ *     y_j = x_j * g_j / sqrt(sum_j(x_j^2) / D + eps),
+ * with g = gamma_q[0..D) for query heads (h < Hq) and gamma_k[0..D) for key
+ * heads.
+ */
+int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
+                    const float *gamma_q, const float *gamma_k, float eps, void *stream);
+
+/*
+ * Layerwise QK-Norm in the SwiftQK form.  Sources: SwiftQK abstract
+ * (newx.sg paper page: under tensor parallelism the normalisation factor of
+ * layerwise QK-Norm depends on the full hidden vector, so ranks exchange only
+ * scalar statistics) and the SwiftQK review (key_machinery: the per-rank
+ * factor is replaced by 1/sqrt((sum_r S_local,r)/H + eps)).  Per token, the
+ * q vector (columns [0, Hq*D), weight gamma_q[0..Hq*D)) and the k vector
+ * (columns [Hq*D, (Hq+Hk)*D), weight gamma_k[0..Hk*D)) are each split into
+ * nshards contiguous head-aligned slices (tensor-parallel split by head, the
+ * lesson's follow-up); each slice's fp32 partial sum of squares S_r is
+ * formed from that slice alone, the partials are combined as scalars, and
+ * every element is scaled by 1/sqrt(S / L + eps) with L the FULL vector
+ * length.  nshards is 1, 2, 4 or 8 and must divide both Hq and Hk.  All
+ * shards run inside one kernel on one GPU; there is no cross-GPU traffic.
+ * The reduction is a fixed tree whose subtrees are the shards, so the output
+ * is bit-identical for every valid nshards.  A token's Q+K span must fit one
+ * thread block: (Hq + Hk) * D * sizeof(element) <= 64 KiB for bf16 and
+ * <= 128 KiB for fp32, else QKN_ERR_UNSUPPORTED.
+ */
+int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
+                     const float *gamma_q, const float *gamma_k, float eps, int nshards,
+                     void *stream);
+
+/* Static English text for a qkn_status value (never NULL). */
+const char *qknorm_status_string(int status);
+
+/* cudaError_t of the calling thread's last QKN_ERR_CUDA (0 if none). */
+int qknorm_last_cuda_error(void);
+
+/* ABI version: 100 * major + minor. */
+int qknorm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNORM_H */

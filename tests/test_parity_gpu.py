@@ -1,0 +1,214 @@
+"""GPU parity: libqknorm.so (through its C ABI) against the float64 oracle.
+
+Every case draws the same seeded input for both sides.  Sizes the oracle
+finishes in seconds are compared element by element over the whole buffer
+(several tiles plus ragged tails); the full-size workloads are compared on
+sampled tokens (random ones, the first and last, and every all-zero or
+outlier row found), which the oracle computes one token at a time.
+Tolerances are in ``tests/gpu_util.py``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attention_qk_norm_b200 as qkn
+from attention_qk_norm_b200 import synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 3
+GUARD_VALUE = -7.25
+
+
+def run(kind, qkv, c, gq, gk, nshards=1, stream=None):
+    if kind == "per_head":
+        qkn.qknorm_per_head(qkv, c.Hq, c.Hk, c.D, gq, gk, c.eps, row_stride=c.row_stride,
+                            stream=stream)
+    else:
+        qkn.qknorm_layerwise(qkv, c.Hq, c.Hk, c.D, gq, gk, c.eps, nshards=nshards,
+                             row_stride=c.row_stride, stream=stream)
+
+
+def full_parity(case, kind, nshards=1, what=""):
+    full, gq, gk = gu.to_device(case, extra_rows=GUARD)
+    run(kind, full[: case.T], case, gq, gk, nshards)
+    torch.cuda.synchronize()
+    out = gu.stored_bits(full)
+    want = gu.oracle_out(case, kind, case.qkv, case.T)
+    qk = (case.Hq + case.Hk) * case.D
+    err = gu.check(out[: case.T], want, case.qkv, case.dtype, qk, what)
+    guard = out[case.T:]
+    ref = gu.stored_bits(torch.full((1,), GUARD_VALUE, dtype=full.dtype))[0]
+    assert np.all(guard == ref), "%s: wrote past the last row" % what
+    return out[: case.T], err
+
+
+# ------------------------------------------------------------------ configs --
+def test_smoke_config():
+    c = synth.make_case(**synth.SMOKE)
+    full_parity(c, "per_head", what="smoke")
+
+
+@pytest.mark.parametrize("H", synth.SWEEP_HEADS)
+@pytest.mark.parametrize("T", synth.SWEEP_T + (3, 257, 1000))
+def test_per_head_sweep(H, T):
+    c = synth.sweep_case(H, T)
+    assert c.Hk == 0 and c.row_stride == H * 128
+    full_parity(c, "per_head", what="sweep H=%d T=%d" % (H, T))
+
+
+@pytest.mark.parametrize("T", (1, 64, 1024, 4096, 3001))
+def test_gqa_fused(T):
+    c = synth.make_case(T, seed=synth.GQA_SEED + T, **synth.GQA)
+    assert c.row_stride == 6144
+    full_parity(c, "per_head", what="gqa T=%d" % T)
+
+
+@pytest.mark.parametrize("T", (1, 16, 256, 4096, 1000))
+def test_layerwise(T):
+    c = synth.make_case(T, seed=synth.LAYERWISE_SEED + T, **synth.LAYERWISE)
+    outs = [full_parity(c, "layerwise", n, what="layerwise T=%d n=%d" % (T, n))[0]
+            for n in synth.LAYERWISE_NSHARDS]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0]), "layerwise output depends on nshards"
+
+
+@pytest.mark.parametrize("dtype", synth.STRESS_DTYPES)
+@pytest.mark.parametrize("D", synth.STRESS_D)
+@pytest.mark.parametrize("eps", synth.STRESS_EPS)
+def test_stress_small(dtype, D, eps):
+    kw = dict(synth.STRESS, T=1037)
+    c = synth.make_case(D=D, dtype=dtype, eps=eps, seed=synth.STRESS_SEED + D, **kw)
+    full_parity(c, "per_head", what="stress per-head %s D=%d" % (dtype, D))
+    lw = synth.make_case(D=D, dtype=dtype, eps=eps, seed=synth.STRESS_SEED + D, layerwise=True,
+                         **kw)
+    a, _ = full_parity(lw, "layerwise", 8, what="stress layerwise %s D=%d" % (dtype, D))
+    b, _ = full_parity(lw, "layerwise", 1, what="stress layerwise %s D=%d" % (dtype, D))
+    assert np.array_equal(a, b)
+
+
+# --------------------------------------------------- full sizes, sampled --
+def sampled_parity(d, kind, nshards_list=(1,), n_random=256, seed=0):
+    qkv = d["qkv"]
+    c = gu.Sampled(d)
+    qk = (c.Hq + c.Hk) * c.D
+    idx = gu.sample_tokens(qkv, qk, n_random, seed)
+    x_s = gu.stored_bits(qkv[idx])
+    want = gu.oracle_out(c, kind, x_s, int(idx.numel()))
+    first = None
+    for n in nshards_list:
+        buf = qkv.clone() if len(nshards_list) > 1 else qkv
+        run(kind, buf, c, d["gamma_q"], d["gamma_k"], n)
+        torch.cuda.synchronize()
+        gu.check(gu.stored_bits(buf[idx]), want, x_s, c.dtype, qk, "%s n=%d" % (kind, n))
+        bits = buf.view(torch.int16) if buf.dtype == torch.bfloat16 else buf.view(torch.int32)
+        if first is None:
+            first = bits
+        else:
+            assert torch.equal(bits, first), "output depends on nshards"
+        del buf
+
+
+def test_sweep_full_size_h48_t4096_sampled():
+    d = synth.make_case_torch(4096, 48, 0, 128, device="cuda", seed=7, eps=1e-6)
+    sampled_parity(d, "per_head")
+
+
+def test_gqa_full_size_sampled():
+    T = synth.GQA_T[-1]
+    d = synth.make_case_torch(T, device="cuda", seed=synth.GQA_SEED, **synth.GQA)
+    sampled_parity(d, "per_head")
+
+
+def test_layerwise_full_size_sampled():
+    T = synth.LAYERWISE_T[-1]
+    d = synth.make_case_torch(T, device="cuda", seed=synth.LAYERWISE_SEED, **synth.LAYERWISE)
+    sampled_parity(d, "layerwise", synth.LAYERWISE_NSHARDS)
+
+
+@pytest.mark.parametrize("dtype", synth.STRESS_DTYPES)
+@pytest.mark.parametrize("D", synth.STRESS_D)
+@pytest.mark.parametrize("eps", synth.STRESS_EPS)
+def test_stress_full_size_sampled(dtype, D, eps):
+    d = synth.make_case_torch(D=D, dtype=dtype, eps=eps, device="cuda",
+                              seed=synth.STRESS_SEED + D, **synth.STRESS)
+    sampled_parity(d, "per_head", seed=D)
+    del d
+    d = synth.make_case_torch(D=D, dtype=dtype, eps=eps, device="cuda", layerwise=True,
+                              seed=synth.STRESS_SEED + D, **synth.STRESS)
+    sampled_parity(d, "layerwise", (1, 8), n_random=128, seed=D)
+    del d
+    torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------- edge cases --
+def test_empty_input_is_a_no_op():
+    x = torch.empty((0, 2560), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(128, device="cuda")
+    qkn.qknorm_per_head(x, 16, 2, 128, g, g, 1e-6)
+    qkn.qknorm_layerwise(x, 16, 2, 128, torch.ones(2048, device="cuda"),
+                         torch.ones(256, device="cuda"), 1e-6, nshards=2)
+
+
+@pytest.mark.parametrize("dtype", (synth.BF16, synth.FP32))
+@pytest.mark.parametrize("D", synth.STRESS_D)
+def test_padded_rows_and_key_only(dtype, D):
+    es = 2 if dtype == synth.BF16 else 4
+    pad = 48 // es  # 48 bytes of padding keeps rows 16-byte aligned
+    c = synth.make_case(37, 3, 2, D, dtype=dtype, seed=11, row_stride=(3 + 4) * D + pad)
+    full_parity(c, "per_head", what="padded")
+    c = synth.make_case(9, 0, 3, D, dtype=dtype, seed=12)
+    full_parity(c, "per_head", what="key heads only")
+    c = synth.make_case(9, 2, 2, D, dtype=dtype, seed=13, row_stride=6 * D + pad,
+                        layerwise=True)
+    full_parity(c, "layerwise", 2, what="layerwise padded")
+
+
+@pytest.mark.parametrize("Hq,Hk,ns", [(40, 8, (1, 2, 4, 8)), (24, 4, (1, 2, 4)), (3, 1, (1,)),
+                                      (6, 2, (1, 2)), (64, 8, (1, 8)), (1, 0, (1,))])
+def test_layerwise_head_counts(Hq, Hk, ns):
+    c = synth.make_case(23, Hq, Hk, 128, seed=Hq * 10 + Hk, layerwise=True)
+    outs = [full_parity(c, "layerwise", n, what="Hq=%d Hk=%d n=%d" % (Hq, Hk, n))[0] for n in ns]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
+def test_zero_eps_on_nonzero_rows():
+    c = synth.make_case(64, 4, 2, 128, seed=21, eps=0.0)
+    full_parity(c, "per_head", what="eps=0")
+    c = synth.make_case(64, 4, 2, 128, seed=22, eps=0.0, layerwise=True)
+    full_parity(c, "layerwise", 2, what="eps=0 layerwise")
+
+
+def test_side_stream_and_repeatability():
+    c = synth.make_case(777, 32, 8, 128, seed=31, scale="lognormal")
+    a, gq, gk = gu.to_device(c)
+    b = a.clone()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        run("per_head", a, c, gq, gk, stream=s)
+    s.synchronize()
+    run("per_head", b, c, gq, gk)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_errors_leave_buffer_untouched():
+    c = synth.make_case(8, 16, 2, 128, seed=41)
+    full, gq, gk = gu.to_device(c)
+    before = full.clone()
+    with pytest.raises(qkn.QKNormError) as e:
+        # a view that starts 8 bytes into the buffer: misaligned base pointer
+        qkn.qknorm_per_head(full[:, 4:], 16, 2, 128, gq, gk, 1e-6, row_stride=2560)
+    assert e.value.status == -3
+    with pytest.raises(qkn.QKNormError) as e:
+        qkn.qknorm_layerwise(full, 16, 2, 128, gq, gk, 1e-6, nshards=4)
+    assert e.value.status == -4
+    wide = torch.zeros((1, (128 + 16) * 256), dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(128 * 256, device="cuda")
+    with pytest.raises(qkn.QKNormError) as e:
+        qkn.qknorm_layerwise(wide, 128, 8, 256, g, g, 1e-6)
+    assert e.value.status == -5
+    torch.cuda.synchronize()
+    assert torch.equal(full.view(torch.int16), before.view(torch.int16))
