@@ -11,17 +11,23 @@
 // from the SwiftQK review, core_discovery): one sub-warp of LPR lanes owns a
 // (token, head) row of D elements.  Each lane holds D*sizeof/16/LPR 16-byte
 // vectors of the row, sums squares in fp32, and the sub-warp reduces with
-// xor shuffles.  Every thread keeps U rows in flight per iteration and its
+// xor shuffles.  Every thread keeps four rows in flight per iteration and its
 // slice of gamma_q / gamma_k in registers for the whole launch.
 //
-// Layerwise (SwiftQK abstract; review key_machinery): one thread block owns
-// a token at a time (persistent, grid-stride over tokens).  Each head's
-// partial sum of squares goes to shared memory; per vector (q, k), one warp
-// forms each emulated shard's fp32 partial from its own heads only, stores
-// the n shard scalars to shared memory (the scalar exchange), and combines
-// them; then every thread scales its registers by the vector's inverse RMS.
-// The next token's data is loaded before the current token's reduction so
-// that the loads overlap the barriers.
+// Layerwise (SwiftQK abstract; review key_machinery): a persistent block
+// walks tokens with a grid stride.  Each thread copies its 16-byte vectors of
+// the next token into a two-stage shared-memory ring with cp.async while it
+// works on the current one.  The per-head partial sums of squares meet in
+// shared memory behind one barrier; then each warp forms every emulated
+// shard's fp32 partial from that shard's heads alone and combines the shard
+// scalars, and every thread scales its vectors, re-read from the ring, by the
+// inverse RMS of its vector.
+//
+// Both kernels are launched with programmatic dependent launch: they wait on
+// griddepcontrol.wait before their first global memory access, so a kernel
+// earlier in the stream always finishes first, and they allow the next
+// kernel to be scheduled as soon as all of their blocks are resident.  No
+// kernel here waits on another block, so none can hang.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -36,7 +42,6 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxShards = 8;
 
 // ---------------------------------------------------------------- vectors --
 template <typename TS>
@@ -112,8 +117,32 @@ __device__ __forceinline__ float group_sum(float s)
     return s;
 }
 
+// Programmatic dependent launch: wait for the grids this one depends on (all
+// their memory operations visible), then let dependents be scheduled.
+__device__ __forceinline__ void pdl_wait_then_release()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
+// cp.async (16 bytes, L2 only) into shared memory, in commit groups.  Each
+// thread waits only for its own groups (cp.async.wait_group), which the
+// hardware completes; there is no spin loop.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- per-head --
 constexpr int kPerHeadThreads = 256;
+constexpr int kPerHeadRowsInFlight = 4;
 
 template <typename TS, int D, int U>
 __global__ void __launch_bounds__(kPerHeadThreads)
@@ -129,6 +158,7 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, uint64_t rows, uin
     constexpr int kEPL = kVPL * kVec;              // elements per lane per row
     static_assert(32 % kLPR == 0 && kNV % kLPR == 0, "row must map onto a sub-warp");
 
+    pdl_wait_then_release();
     const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const uint32_t lane = (uint32_t)(tid % kLPR);
     const uint64_t group = tid / kLPR;
@@ -210,93 +240,66 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, uint64_t rows, uin
 }
 
 // --------------------------------------------------------------- layerwise --
-// Shared-memory scratch of one block, laid out after the per-head partials:
-//   part[heads]          per-head fp32 partial sums of squares
-//   tree[heads]          leaves / partial sums of the fixed reduction tree
-//   shard[2][8]          the emulated ranks' scalar partials (q, k)
-//   rinv[2]              inverse RMS of the q and k vectors
-struct LayerwiseSmem {
-    float *part, *tree, *shard, *rinv;
-    __device__ LayerwiseSmem(float *base, int heads)
-        : part(base), tree(base + heads), shard(base + 2 * heads),
-          rinv(base + 2 * heads + 2 * kMaxShards) {}
-};
+constexpr int kLayerwiseStages = 2;
 
-// One warp: inverse RMS of one vector of `nh` heads from their partials.
+// Inverse RMS of one vector of `nh` heads from their partials part[0..nh),
+// computed by one whole warp; every lane returns the same value.
 //
-// The reduction tree is fixed by nh alone: nh = m * 2^k with m odd; leaf i
-// is the in-order sum of heads [i*m, (i+1)*m), and the 2^k leaves are summed
-// pairwise (adjacent pairs first).  A shard of nh/n heads (n a power of two
-// dividing nh) is then exactly one subtree, so its partial S_r is formed from
-// its own heads only; the n scalars are written to shared memory and combined
-// pairwise, which finishes the same tree.  Hence the result does not depend
-// on n, bit for bit.
-__device__ __forceinline__ void combine_vector(const float *part, float *tree, float *shard,
-                                               float *rinv_out, int nh, int nshards,
-                                               float len, float eps, int lane)
+// The reduction tree is fixed by nh alone.  Let p be the largest power of two
+// dividing nh and u = min(p, 32) the lanes used: lane i sums heads
+// [i*c, (i+1)*c) in order (c = nh/u), then xor butterflies join lanes at
+// distance 1, 2, 4, ...  With n shards (n a power of two dividing nh, so
+// n <= u), shard r holds exactly lanes [r*u/n, (r+1)*u/n): the butterflies
+// below distance u/n form each shard's partial S_r from that shard's heads
+// only, and the remaining ones are the scalar combine of S_0..S_{n-1}.  So
+// the result does not depend on n, bit for bit.
+__device__ __forceinline__ float warp_rinv(const float *part, int nh, int nshards, float len,
+                                           float eps, int lane)
 {
-    if (nh == 0) return;
-    int m = nh;
-    while ((m & 1) == 0) m >>= 1;
-    const int leaves = nh / m;
-    for (int i = lane; i < leaves; i += 32) {
-        float s = 0.f;
-        for (int j = 0; j < m; ++j) s += part[i * m + j];
-        tree[i] = s;
-    }
-    __syncwarp();
-    const int per_shard = leaves / nshards;  // leaves in one shard's subtree
-    for (int w = 1; w < per_shard; w *= 2) {
-        for (int i = lane * 2 * w; i < leaves; i += 64 * w) tree[i] += tree[i + w];
-        __syncwarp();
-    }
-    // Scalar exchange: shard r publishes S_r; the combine reads only these.
-    if (lane < nshards) shard[lane] = tree[lane * per_shard];
-    __syncwarp();
-    if (lane == 0) {
-        float s[kMaxShards];
-        for (int r = 0; r < nshards; ++r) s[r] = shard[r];
-        for (int w = 1; w < nshards; w *= 2)
-            for (int r = 0; r < nshards; r += 2 * w) s[r] += s[r + w];
-        *rinv_out = rsqrtf(s[0] / len + eps);
-    }
+    if (nh == 0) return 0.f;
+    const int p2 = nh & (-nh);
+    const int used = p2 < 32 ? p2 : 32;
+    const int c = nh / used;
+    float v = 0.f;
+    if (lane < used)
+        for (int j = 0; j < c; ++j) v += part[lane * c + j];
+    const int per_shard = used / nshards;
+    for (int o = 1; o < per_shard; o <<= 1)  // rank-local partial S_r
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = per_shard; o < used; o <<= 1)  // combine of the shard scalars
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    v = __shfl_sync(0xffffffffu, v, 0);
+    return rsqrtf(v / len + eps);
 }
 
-// Block-size ceiling by elements per thread, so that one token's block fits
-// the 64K-register file without spills.  With gamma held in registers:
-// 1024 threads up to 8 elements, 768 at 16, 512 at 32.  The variant that
-// reads gamma from L1 at scale time keeps fewer registers: 1024 up to 16
-// elements, 768 at 32.
-constexpr int layerwise_max_threads(int ept, bool gamma_regs)
-{
-    return gamma_regs ? (ept <= 8 ? 1024 : (ept <= 16 ? 768 : 512)) : (ept <= 16 ? 1024 : 768);
-}
-
+// A block of roundup32(heads * NV / VPT) threads; thread (h, l) owns vectors
+// l, l + LPH, ... of head h (LPH = NV / VPT lanes per head).  Dynamic shared
+// memory: kLayerwiseStages token stages of span = heads*D*sizeof(TS) bytes,
+// then two buffers of `heads` fp32 head partials (alternating per token).
 template <typename TS, int D, int VPT, bool kGammaRegs>
-__global__ void __launch_bounds__(layerwise_max_threads(VPT * Storage<TS>::kVec, kGammaRegs))
-qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq,
-                                     int Hk, int nshards, const float *__restrict__ gamma_q,
-                                     const float *__restrict__ gamma_k, float eps, float len_q,
-                                     float len_k)
+__global__ void __launch_bounds__(1024)
+qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                     int nshards, const float *__restrict__ gamma_q,
+                     const float *__restrict__ gamma_k, float eps, float len_q, float len_k)
 {
     using S = Storage<TS>;
     constexpr int kVec = S::kVec;
-    constexpr int kNV = D / kVec;    // 16-byte vectors per head
-    constexpr int kLPH = kNV / VPT;  // threads per head
-    constexpr int kEPT = VPT * kVec; // elements per thread
+    constexpr int kNV = D / kVec;     // 16-byte vectors per head
+    constexpr int kLPH = kNV / VPT;   // threads per head
+    constexpr int kEPT = VPT * kVec;  // elements per thread
+    constexpr int NST = kLayerwiseStages;
     static_assert(kNV % VPT == 0 && 32 % kLPH == 0, "head must map onto a sub-warp");
 
-    extern __shared__ float smem_raw[];
+    extern __shared__ __align__(16) unsigned char smem[];
     const int heads = Hq + Hk;
-    LayerwiseSmem sm(smem_raw, heads);
-
+    const int span = heads * D * (int)sizeof(TS);
+    float *part = reinterpret_cast<float *>(smem + (size_t)NST * span);
     const int h = threadIdx.x / kLPH;
     const int l = threadIdx.x % kLPH;
     const bool active = h < heads;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int nwarps = blockDim.x / 32;
+    const int lane = threadIdx.x % 32;
 
-    // Fixed columns of this thread: vectors l, l + LPH, ... of head h.
+    pdl_wait_then_release();
     const float *gb = !active ? gamma_q
                       : (h < Hq ? gamma_q + (int64_t)h * D : gamma_k + (int64_t)(h - Hq) * D);
     float g[kGammaRegs ? kEPT : 1];
@@ -312,46 +315,49 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         }
     }
     const int64_t col0 = (int64_t)h * D;
-
-    uint4 cur[VPT], nxt[VPT];
+    // Each thread copies, and later reads, only its own vectors of a stage.
+    auto fetch = [&](int64_t tok, int st) {
+        if (active && tok < T) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(qkv + tok * row_stride + col0);
+            unsigned char *dst = smem + (size_t)st * span + col0 * sizeof(TS);
 #pragma unroll
-    for (int v = 0; v < VPT; ++v) cur[v] = nxt[v] = make_uint4(0u, 0u, 0u, 0u);
-    int64_t t = blockIdx.x;
-    if (active && t < T) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(qkv + t * row_stride + col0);
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) cur[v] = load_stream(p + l + v * kLPH);
-    }
-    for (; t < T; t += gridDim.x) {
-        const int64_t tn = t + gridDim.x;
-        if (active && tn < T) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(qkv + tn * row_stride + col0);
-#pragma unroll
-            for (int v = 0; v < VPT; ++v) nxt[v] = load_stream(p + l + v * kLPH);
+            for (int v = 0; v < VPT; ++v) cp_async16(dst + (l + v * kLPH) * 16, src + l + v * kLPH);
         }
-        float f[VPT][kVec];
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int i = 0; i < NST - 1; ++i) fetch(blockIdx.x + (int64_t)i * gridDim.x, i);
+    int st = 0, pb = 0;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        // Refill the stage this thread finished with on the previous token.
+        fetch(t + (int64_t)(NST - 1) * gridDim.x, (st + NST - 1) % NST);
+        cp_async_wait<NST - 1>();
+        const uint4 *sp =
+            reinterpret_cast<const uint4 *>(smem + (size_t)st * span + col0 * sizeof(TS));
         float s = 0.f;
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
-            S::unpack(cur[v], f[v]);
+            float f[kVec];
+            S::unpack(active ? sp[l + v * kLPH] : make_uint4(0u, 0u, 0u, 0u), f);
 #pragma unroll
-            for (int e = 0; e < kVec; ++e) s = fmaf(f[v][e], f[v][e], s);
+            for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
         }
         s = group_sum<kLPH>(s);
-        if (active && l == 0) sm.part[h] = s;
+        // Partials alternate between two buffers: a warp still reading this
+        // token's buffer cannot meet a write of the next token's, which only
+        // starts after the next barrier.
+        float *pp = part + pb * heads;
+        if (active && l == 0) pp[h] = s;
         __syncthreads();
-        if (warp == 0)
-            combine_vector(sm.part, sm.tree, sm.shard, sm.rinv, Hq, nshards, len_q, eps, lane);
-        if (warp == (nwarps > 1 ? 1 : 0))
-            combine_vector(sm.part + Hq, sm.tree + Hq, sm.shard + kMaxShards, sm.rinv + 1, Hk,
-                           nshards, len_k, eps, lane);
-        __syncthreads();
+        const float rq = warp_rinv(pp, Hq, nshards, len_q, eps, lane);
+        const float rk = warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane);
         if (active) {
-            const float rinv = sm.rinv[h < Hq ? 0 : 1];
+            const float rinv = h < Hq ? rq : rk;
             uint4 *p = reinterpret_cast<uint4 *>(qkv + t * row_stride + col0);
 #pragma unroll
             for (int v = 0; v < VPT; ++v) {
-                float o[kVec], gv[kVec];
+                float f[kVec], o[kVec], gv[kVec];
+                S::unpack(sp[l + v * kLPH], f);
                 if constexpr (kGammaRegs) {
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
@@ -359,13 +365,14 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
                     load_gamma<kVec>(gb + (l + v * kLPH) * kVec, gv);
                 }
 #pragma unroll
-                for (int e = 0; e < kVec; ++e) o[e] = f[v][e] * rinv * gv[e];
+                for (int e = 0; e < kVec; ++e) o[e] = f[e] * rinv * gv[e];
                 store_stream(p + l + v * kLPH, S::pack(o));
             }
         }
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) cur[v] = nxt[v];
+        st = (st + 1 == NST) ? 0 : st + 1;
+        pb ^= 1;
     }
+    cp_async_wait<0>();
 }
 
 // ------------------------------------------------------------------- host --
@@ -379,12 +386,13 @@ int cuda_fail(cudaError_t e)
 
 struct DeviceInfo {
     int sms = 0;
+    int smem_optin = 0;  // max dynamic shared memory per block (opt-in)
 };
 
 std::mutex g_dev_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-int device_sms(int *sms)
+int device_info(int *dev_out, DeviceInfo *info)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -392,24 +400,38 @@ int device_sms(int *sms)
     if (dev < 0 || dev >= kMaxDevices) return QKN_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_dev_mu);
     if (g_dev[dev].sms == 0) {
-        int n = 0;
+        int n = 0, smem = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
         g_dev[dev].sms = n;
+        g_dev[dev].smem_optin = smem;
     }
-    *sms = g_dev[dev].sms;
+    *dev_out = dev;
+    *info = g_dev[dev];
     return QKN_OK;
 }
 
-// Resident blocks per SM of one kernel at one block size (cached).
-template <typename Kernel>
-int blocks_per_sm(Kernel k, int threads, size_t smem, int *out)
+// Launch with programmatic stream serialization allowed (see the kernels'
+// griddepcontrol.wait), then report the launch status.
+template <typename... Params, typename... Args>
+int launch_pdl(void (*kern)(Params...), unsigned grid, unsigned threads, size_t smem,
+               cudaStream_t stream, Args... args)
 {
-    int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    *out = n > 0 ? n : 1;
-    return QKN_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -443,7 +465,34 @@ int validate(const void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64
     return QKN_OK;
 }
 
-constexpr int kPerHeadRowsInFlight = 2;
+// Per-kernel, per-device set-up done once: the opt-in dynamic shared-memory
+// limit, and (for kernels without dynamic shared memory) the resident blocks
+// per SM at the block size in use.
+struct KernelCache {
+    std::atomic<int> per_sm[kMaxDevices][33] = {};
+    std::atomic<uint64_t> smem_ready{0};
+};
+
+template <typename Kern>
+int resident_blocks(Kern kern, KernelCache &kc, int dev, const DeviceInfo &info, int threads,
+                    size_t smem, int *out)
+{
+    if (smem > 48 * 1024 && !(kc.smem_ready.load(std::memory_order_acquire) & (1ull << dev))) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            kern, cudaFuncAttributeMaxDynamicSharedMemorySize, info.smem_optin);
+        if (e != cudaSuccess) return cuda_fail(e);
+        kc.smem_ready.fetch_or(1ull << dev, std::memory_order_acq_rel);
+    }
+    const int slot = threads / 32;
+    int n = smem == 0 ? kc.per_sm[dev][slot].load(std::memory_order_relaxed) : 0;
+    if (n == 0) {
+        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (smem == 0) kc.per_sm[dev][slot].store(n, std::memory_order_relaxed);
+    }
+    *out = n;
+    return QKN_OK;
+}
 
 template <typename TS, int D>
 int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
@@ -453,36 +502,39 @@ int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, co
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kLPR = kNV < 32 ? kNV : 32;
     auto kern = qkn_per_head_kernel<TS, D, U>;
-    int sms = 0, per_sm = 0, rc;
-    if ((rc = device_sms(&sms)) != QKN_OK) return rc;
-    static std::atomic<int> cached_per_sm{0};  // same sm_100a image on every device
-    per_sm = cached_per_sm.load(std::memory_order_relaxed);
-    if (per_sm == 0) {
-        if ((rc = blocks_per_sm(kern, kPerHeadThreads, 0, &per_sm)) != QKN_OK) return rc;
-        cached_per_sm.store(per_sm, std::memory_order_relaxed);
-    }
+    static KernelCache kc;
+    int dev = 0, per_sm = 0, rc;
+    DeviceInfo info;
+    if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
+    if ((rc = resident_blocks(kern, kc, dev, info, kPerHeadThreads, 0, &per_sm)) != QKN_OK)
+        return rc;
+    if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
     // Qwen3 gamma is shared by every head: pass nullptr for K when Hk == 0.
     const float *gq_eff = Hq > 0 ? gq : gk;
     const float *gk_eff = Hk > 0 ? gk : nullptr;
     const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
     const uint64_t rows_per_block = (uint64_t)(kPerHeadThreads / kLPR) * U;
     const uint64_t need = (rows + rows_per_block - 1) / rows_per_block;
-    const uint64_t cap = (uint64_t)sms * per_sm;
+    const uint64_t cap = (uint64_t)info.sms * per_sm;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    kern<<<grid, kPerHeadThreads, 0, stream>>>(static_cast<TS *>(qkv), row_stride, rows,
-                                               (uint32_t)(Hq + Hk), (uint32_t)Hq, gq_eff, gk_eff,
-                                               eps);
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
+    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, static_cast<TS *>(qkv), row_stride,
+                      rows, (uint32_t)(Hq + Hk), (uint32_t)Hq, gq_eff, gk_eff, eps);
 }
 
 // A layerwise kernel variant exists when a head splits into whole 16-byte
-// vectors per thread on at most 32 lanes, with at most 32 elements per thread.
+// vectors per thread on at most 32 lanes.  Gamma stays in registers up to 32
+// elements per thread, else it is read through L1 when scaling.
 template <typename TS, int D, int VPT>
 constexpr bool layerwise_vpt_ok()
 {
     constexpr int kNV = D / Storage<TS>::kVec;
-    return kNV % VPT == 0 && kNV / VPT <= 32 && VPT * Storage<TS>::kVec <= 32;
+    return kNV % VPT == 0 && kNV / VPT <= 32;
+}
+
+template <typename TS, int VPT>
+constexpr bool layerwise_gamma_regs()
+{
+    return VPT * Storage<TS>::kVec <= 32;
 }
 
 template <typename TS, int D, int VPT>
@@ -490,47 +542,27 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
                          const float *gq, const float *gk, float eps, int nshards, int threads,
                          cudaStream_t stream)
 {
+    auto kern = qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>()>;
+    static KernelCache kc;
     const int heads = Hq + Hk;
-    constexpr int kEPT = VPT * Storage<TS>::kVec;
-    // Gamma in registers when the block fits that variant, else from L1.
-    auto kern = threads <= layerwise_max_threads(kEPT, true)
-                    ? qkn_layerwise_kernel<TS, D, VPT, true>
-                    : qkn_layerwise_kernel<TS, D, VPT, false>;
-    const bool regs_variant = threads <= layerwise_max_threads(kEPT, true);
-    const size_t smem = (size_t)(2 * heads + 2 * kMaxShards + 2) * sizeof(float);
-    int sms = 0, per_sm = 0, rc;
-    if ((rc = device_sms(&sms)) != QKN_OK) return rc;
-    // Per block size (a multiple of 32 up to 1024): the register-limited
-    // maximum and the resident blocks per SM, both computed once.
-    static std::atomic<int> max_threads[2];
-    static std::atomic<int> cached[2][33];
-    int mt = max_threads[regs_variant].load(std::memory_order_relaxed);
-    if (mt == 0) {
-        cudaFuncAttributes attr;
-        const cudaError_t e = cudaFuncGetAttributes(&attr, kern);
-        if (e != cudaSuccess) return cuda_fail(e);
-        mt = attr.maxThreadsPerBlock;
-        max_threads[regs_variant].store(mt, std::memory_order_relaxed);
-    }
-    if (threads > mt) return QKN_ERR_UNSUPPORTED;
-    per_sm = cached[regs_variant][threads / 32].load(std::memory_order_relaxed);
-    if (per_sm == 0) {
-        if ((rc = blocks_per_sm(kern, threads, smem, &per_sm)) != QKN_OK) return rc;
-        cached[regs_variant][threads / 32].store(per_sm, std::memory_order_relaxed);
-    }
-    const int64_t cap = (int64_t)sms * per_sm;
+    const size_t span = (size_t)heads * D * sizeof(TS);
+    const size_t smem = kLayerwiseStages * span + (size_t)2 * heads * sizeof(float);
+    int dev = 0, per_sm = 0, rc;
+    DeviceInfo info;
+    if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
+    if (smem > (size_t)info.smem_optin) return QKN_ERR_UNSUPPORTED;
+    if ((rc = resident_blocks(kern, kc, dev, info, threads, smem, &per_sm)) != QKN_OK) return rc;
+    if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
+    const int64_t cap = (int64_t)info.sms * per_sm;
     const unsigned grid = (unsigned)(T < cap ? T : cap);
     const float len_q = (float)((int64_t)Hq * D);  // exact: spans are < 2^24 elements
     const float len_k = (float)((int64_t)Hk * D);
-    kern<<<grid, threads, smem, stream>>>(static_cast<TS *>(qkv), row_stride, T, Hq, Hk, nshards,
-                                          gq, gk, eps, len_q, len_k);
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
+    return launch_pdl(kern, grid, threads, smem, stream, static_cast<TS *>(qkv), row_stride, T,
+                      Hq, Hk, nshards, gq, gk, eps, len_q, len_k);
 }
 
-// Vectors per thread: the fewest that keep a token's block within
-// kLayerwiseTargetThreads, else within 1024 threads; at most 32 fp32
-// elements per thread (registers).
+// Vectors per thread: the fewest that keep a token's block within 256
+// threads, else within 1024.
 constexpr int kLayerwiseTargetThreads = 256;
 
 template <typename TS, int D>
@@ -538,15 +570,13 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
                      const float *gk, float eps, int nshards, cudaStream_t stream)
 {
     constexpr int kNV = D / Storage<TS>::kVec;
-    constexpr int kMaxVPT = 32 / Storage<TS>::kVec;  // 4 for bf16, 8 for fp32
     const int64_t heads = Hq + Hk;
     int chosen = 0;
     for (int pass = 0; pass < 2 && chosen == 0; ++pass) {
-        const int64_t limit = pass == 0 ? kLayerwiseTargetThreads : 768;
-        for (int vpt = 1; vpt <= kMaxVPT; vpt *= 2) {
+        const int64_t limit = pass == 0 ? kLayerwiseTargetThreads : 1024;
+        for (int vpt = 1; vpt <= kNV; vpt *= 2) {
             if (kNV % vpt != 0 || kNV / vpt > 32) continue;  // mirrors layerwise_vpt_ok
-            const int64_t threads = ((heads * (kNV / vpt) + 31) / 32) * 32;
-            if (threads <= limit) {
+            if (((heads * (kNV / vpt) + 31) / 32) * 32 <= limit) {
                 chosen = vpt;
                 break;
             }
@@ -554,30 +584,24 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
     }
     if (chosen == 0) return QKN_ERR_UNSUPPORTED;
     const int threads = (int)(((heads * (kNV / chosen) + 31) / 32) * 32);
+#define QKN_LW_CASE(V)                                                                         \
+    case V:                                                                                    \
+        if constexpr (layerwise_vpt_ok<TS, D, V>())                                            \
+            return launch_layerwise_vpt<TS, D, V>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,     \
+                                                  nshards, threads, stream);                   \
+        break;
     switch (chosen) {
-    case 1:
-        if constexpr (layerwise_vpt_ok<TS, D, 1>())
-            return launch_layerwise_vpt<TS, D, 1>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
-                                                  nshards, threads, stream);
-        break;
-    case 2:
-        if constexpr (layerwise_vpt_ok<TS, D, 2>())
-            return launch_layerwise_vpt<TS, D, 2>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
-                                                  nshards, threads, stream);
-        break;
-    case 4:
-        if constexpr (layerwise_vpt_ok<TS, D, 4>())
-            return launch_layerwise_vpt<TS, D, 4>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
-                                                  nshards, threads, stream);
-        break;
-    case 8:
-        if constexpr (layerwise_vpt_ok<TS, D, 8>())
-            return launch_layerwise_vpt<TS, D, 8>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
-                                                  nshards, threads, stream);
-        break;
+        QKN_LW_CASE(1)
+        QKN_LW_CASE(2)
+        QKN_LW_CASE(4)
+        QKN_LW_CASE(8)
+        QKN_LW_CASE(16)
+        QKN_LW_CASE(32)
+        QKN_LW_CASE(64)
     default:
         break;
     }
+#undef QKN_LW_CASE
     return QKN_ERR_UNSUPPORTED;
 }
 

@@ -64,7 +64,7 @@ typedef enum {
     QKN_ERR_SHAPE = -2,       /* negative sizes, no heads, row_stride < W       */
     QKN_ERR_ALIGN = -3,       /* qkv, gamma or row_stride bytes not 16-aligned  */
     QKN_ERR_NSHARDS = -4,     /* nshards not in {1,2,4,8} or not dividing heads */
-    QKN_ERR_UNSUPPORTED = -5, /* dtype or head_dim not built, row too wide      */
+    QKN_ERR_UNSUPPORTED = -5, /* dtype or head_dim not built, token too wide    */
     QKN_ERR_CUDA = -6,        /* CUDA runtime error on this call                */
     QKN_ERR_EPS = -7          /* eps negative or not finite                     */
 } qkn_status;
@@ -98,9 +98,11 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
  * length.  nshards is 1, 2, 4 or 8 and must divide both Hq and Hk.  All
  * shards run inside one kernel on one GPU; there is no cross-GPU traffic.
  * The reduction is a fixed tree whose subtrees are the shards, so the output
- * is bit-identical for every valid nshards.  A token's Q+K span must fit one
- * thread block: (Hq + Hk) * D * sizeof(element) <= 64 KiB for bf16 and
- * <= 128 KiB for fp32, else QKN_ERR_UNSUPPORTED.
+ * is bit-identical for every valid nshards.  One thread block works on one
+ * token at a time and keeps two tokens staged in shared memory, so the Q+K
+ * span must satisfy 2 * (Hq + Hk) * D * sizeof(element) + 8 * (Hq + Hk)
+ * <= the device's opt-in shared memory per block (227 KiB on B200), else
+ * QKN_ERR_UNSUPPORTED.
  */
 int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
                      const float *gamma_q, const float *gamma_k, float eps, int nshards,

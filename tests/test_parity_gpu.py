@@ -205,7 +205,8 @@ def test_errors_leave_buffer_untouched():
     with pytest.raises(qkn.QKNormError) as e:
         qkn.qknorm_layerwise(full, 16, 2, 128, gq, gk, 1e-6, nshards=4)
     assert e.value.status == -4
-    wide = torch.zeros((1, (128 + 16) * 256), dtype=torch.bfloat16, device="cuda")
+    # 136 fp32 heads of 256: two staged tokens need 272 KiB of shared memory
+    wide = torch.zeros((1, (128 + 16) * 256), dtype=torch.float32, device="cuda")
     g = torch.ones(128 * 256, device="cuda")
     with pytest.raises(qkn.QKNormError) as e:
         qkn.qknorm_layerwise(wide, 128, 8, 256, g, g, 1e-6)
