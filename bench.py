@@ -527,6 +527,33 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_CASES = {
+    "per_head": dict(HEADLINE),
+    "gqa": dict(kind="per_head", T=16384, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6, nshards=1,
+                scale="lognormal", seed=1002),
+    "layerwise": dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
+                      nshards=8, seed=1003),
+}
+
+
+def run_profile(args):
+    """A few plain launches of one workload, for a profiler to capture: no
+    graphs, no timing, no sweep.  ``--profile-T`` overrides the token count."""
+    import torch
+
+    w = dict(PROFILE_CASES[args.profile])
+    if args.profile_T:
+        w["T"] = args.profile_T
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    wl = Workload(w, device, l2_bytes=0)  # one buffer; profilers flush caches themselves
+    for _ in range(args.warmup + args.steps):
+        wl.launch()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "T": w["T"], "launches": args.warmup + args.steps,
+                      "bytes_per_launch": workload_bytes(w)}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -537,11 +564,16 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true", help="skip the T / workload sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=sorted(PROFILE_CASES),
+                    help="only launch one workload's kernel (for ncu captures)")
+    ap.add_argument("--profile-T", type=int, default=0)
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.steps < 1:
         ap.error("--steps must be >= 1")
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -1,0 +1,69 @@
+"""Multi-process host logic of bench.py on CPU (gloo, world size 2).
+
+QK-Norm tokens are independent, so ranks need no collective on the data
+path; the only cross-rank steps are the barrier around the timed region
+and the max over ranks of the elapsed time.  These run here as gloo ranks.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+
+    r, w, _ = bench.dist_init()
+    assert (r, w) == (rank, world) and dist.get_backend() == "gloo"
+    bench.barrier(w)
+    local_ms = 10.0 + 5.0 * rank
+    got = bench.max_over_ranks(local_ms, w)
+    lo, hi = bench.shard_units(1001, w, r)
+    q.put((rank, got, lo, hi))
+    bench.barrier(w)
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_barrier_and_max():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [o[1] for o in out] == [15.0, 15.0]  # max over ranks, seen by every rank
+    spans = [(o[2], o[3]) for o in out]
+    assert spans == [(0, 501), (501, 1001)]
+
+
+@pytest.mark.parametrize("total,world", [(0, 2), (7, 3), (4096, 8), (5, 8)])
+def test_shard_units_partition(total, world):
+    spans = [bench.shard_units(total, world, r) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == total
+    for (a, b), (c, d) in zip(spans, spans[1:]):
+        assert b == c
+    sizes = [b - a for a, b in spans]
+    assert max(sizes) - min(sizes) <= 1
+
+
+def test_algorithmic_bytes():
+    w = dict(bench.HEADLINE)
+    assert bench.workload_bytes(w) == 2 * 4096 * 48 * 128 * 2 + 128 * 4
+    lw = dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16")
+    assert bench.workload_bytes(lw) == 2 * 8192 * 40 * 128 * 2 + 40 * 128 * 4
