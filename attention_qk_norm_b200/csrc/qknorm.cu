@@ -11,17 +11,17 @@
 // from the SwiftQK review, core_discovery): one sub-warp of LPR lanes owns a
 // (token, head) row of D elements.  Each lane holds D*sizeof/16/LPR 16-byte
 // vectors of the row, sums squares in fp32, and the sub-warp reduces with
-// xor shuffles.  Every thread keeps four rows in flight per iteration and its
+// xor shuffles.  Every thread keeps two rows in flight per iteration and its
 // slice of gamma_q / gamma_k in registers for the whole launch.
 //
 // Layerwise (SwiftQK abstract; review key_machinery): a persistent block
 // walks tokens with a grid stride.  Each thread copies its 16-byte vectors of
 // the next token into a two-stage shared-memory ring with cp.async while it
 // works on the current one.  The per-head partial sums of squares meet in
-// shared memory behind one barrier; then each warp forms every emulated
-// shard's fp32 partial from that shard's heads alone and combines the shard
-// scalars, and every thread scales its vectors, re-read from the ring, by the
-// inverse RMS of its vector.
+// shared memory behind one barrier; then each warp, for the vectors (q, k)
+// its threads hold, forms every emulated shard's fp32 partial from that
+// shard's heads alone and combines the shard scalars, and every thread scales
+// its vectors, re-read from the ring, by the inverse RMS of its vector.
 //
 // Both kernels are launched with programmatic dependent launch: they wait on
 // griddepcontrol.wait before their first global memory access, so a kernel
@@ -142,11 +142,24 @@ __device__ __forceinline__ void cp_async_wait()
 
 // ---------------------------------------------------------------- per-head --
 constexpr int kPerHeadThreads = 256;
-constexpr int kPerHeadRowsInFlight = 4;
+constexpr int kPerHeadRowsInFlight = 2;
+// Resident 256-thread blocks per SM that the register budget must allow:
+// six (40 registers) for the single-weight loop with one vector per lane and
+// row, five (48) with both weights, four (64) with two vectors per lane.
+// Each fits without spilling.
+template <typename TS, int D, bool kHasK>
+constexpr int per_head_min_blocks()
+{
+    return D / Storage<TS>::kVec > 32 ? 4 : (kHasK ? 5 : 6);
+}
 
-template <typename TS, int D, int U>
-__global__ void __launch_bounds__(kPerHeadThreads)
-qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, uint64_t rows, uint32_t heads,
+// Rows are visited with a grid stride: thread group g takes rows g, g + G,
+// g + 2G, ... (G groups in the grid), U at a time.  The (token, head) pair of
+// each of its U rows is found once by division and then advanced by the fixed
+// step U*G with an add and one wrap, so the loop does no integer division.
+template <typename TS, int D, int U, bool kHasK>
+__global__ void __launch_bounds__(kPerHeadThreads, (per_head_min_blocks<TS, D, kHasK>()))
+qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_t heads,
                     uint32_t Hq, const float *__restrict__ gamma_q,
                     const float *__restrict__ gamma_k, float eps)
 {
@@ -165,51 +178,45 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, uint64_t rows, uin
     const uint64_t ngroups = ((uint64_t)gridDim.x * blockDim.x) / kLPR;
 
     // This lane's columns are fixed: vectors lane, lane + LPR, ... of a row.
-    float gq[kEPL], gk[kEPL];
+    float gq[kEPL], gk[kHasK ? kEPL : 1];
 #pragma unroll
     for (int v = 0; v < kVPL; ++v) {
         const int col = (lane + v * kLPR) * kVec;
-        float tq[kVec], tk[kVec];
+        float tq[kVec];
         load_gamma<kVec>(gamma_q + col, tq);
-        if (gamma_k != nullptr) load_gamma<kVec>(gamma_k + col, tk);
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) {
-            gq[v * kVec + e] = tq[e];
-            gk[v * kVec + e] = gamma_k != nullptr ? tk[e] : tq[e];
+        for (int e = 0; e < kVec; ++e) gq[v * kVec + e] = tq[e];
+        if constexpr (kHasK) {
+            float tk[kVec];
+            load_gamma<kVec>(gamma_k + col, tk);
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) gk[v * kVec + e] = tk[e];
         }
     }
 
-    const bool small = rows <= 0xffffffffull;
+    int64_t t[U];
+    uint32_t h[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+        const uint64_t r = (uint64_t)k * ngroups + group;
+        t[k] = (int64_t)(r / heads);
+        h[k] = (uint32_t)(r - (uint64_t)t[k] * heads);
+    }
     const uint64_t step = ngroups * U;
+    const int64_t dt = (int64_t)(step / heads);
+    const uint32_t dh = (uint32_t)(step - (uint64_t)dt * heads);
+    const uint64_t rows = (uint64_t)T * heads;
     // The trip count is the same for every thread, so whole warps reach each
     // shuffle together; rows past the end contribute zeros and store nothing.
     for (uint64_t base = 0; base < rows; base += step) {
         uint4 x[U][kVPL];
         uint4 *ptr[U];
-        bool is_q[U];
 #pragma unroll
         for (int k = 0; k < U; ++k) {
-            const uint64_t r = base + (uint64_t)k * ngroups + group;
-            ptr[k] = nullptr;
-            is_q[k] = true;
-            if (r < rows) {
-                uint64_t t, h;
-                if (small) {
-                    const uint32_t r32 = (uint32_t)r;
-                    t = r32 / heads;
-                    h = r32 - (uint32_t)t * heads;
-                } else {
-                    t = r / heads;
-                    h = r - t * heads;
-                }
-                is_q[k] = h < Hq;
-                ptr[k] = reinterpret_cast<uint4 *>(qkv + (int64_t)t * row_stride + (int64_t)h * D);
+            ptr[k] = reinterpret_cast<uint4 *>(qkv + t[k] * row_stride + (int64_t)h[k] * D) + lane;
 #pragma unroll
-                for (int v = 0; v < kVPL; ++v) x[k][v] = load_stream(ptr[k] + lane + v * kLPR);
-            } else {
-#pragma unroll
-                for (int v = 0; v < kVPL; ++v) x[k][v] = make_uint4(0u, 0u, 0u, 0u);
-            }
+            for (int v = 0; v < kVPL; ++v)
+                x[k][v] = t[k] < T ? load_stream(ptr[k] + v * kLPR) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int k = 0; k < U; ++k) {
@@ -223,17 +230,25 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, uint64_t rows, uin
             }
             s = group_sum<kLPR>(s);
             const float rinv = rsqrtf(s / (float)D + eps);
-            if (ptr[k] != nullptr) {
+            if (t[k] < T) {
+                const bool is_q = !kHasK || h[k] < Hq;
 #pragma unroll
                 for (int v = 0; v < kVPL; ++v) {
                     float o[kVec];
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) {
-                        const float g = is_q[k] ? gq[v * kVec + e] : gk[v * kVec + e];
+                        float g = gq[v * kVec + e];
+                        if constexpr (kHasK) g = is_q ? g : gk[v * kVec + e];
                         o[e] = f[v][e] * rinv * g;
                     }
-                    store_stream(ptr[k] + lane + v * kLPR, S::pack(o));
+                    store_stream(ptr[k] + v * kLPR, S::pack(o));
                 }
+            }
+            h[k] += dh;
+            t[k] += dt;
+            if (h[k] >= heads) {
+                h[k] -= heads;
+                t[k] += 1;
             }
         }
     }
@@ -298,6 +313,12 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     const int l = threadIdx.x % kLPH;
     const bool active = h < heads;
     const int lane = threadIdx.x % 32;
+    // Heads of this warp's threads; a warp computes only the inverse RMS of
+    // the vectors it holds (warp-uniform, so whole warps shuffle together).
+    const int warp_first_head = (threadIdx.x & ~31) / kLPH;
+    const int warp_last_head = (threadIdx.x | 31) / kLPH;
+    const bool need_q = warp_first_head < Hq;
+    const bool need_k = Hk > 0 && warp_last_head >= Hq;
 
     pdl_wait_then_release();
     const float *gb = !active ? gamma_q
@@ -349,8 +370,8 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         float *pp = part + pb * heads;
         if (active && l == 0) pp[h] = s;
         __syncthreads();
-        const float rq = warp_rinv(pp, Hq, nshards, len_q, eps, lane);
-        const float rk = warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane);
+        const float rq = need_q ? warp_rinv(pp, Hq, nshards, len_q, eps, lane) : 0.f;
+        const float rk = need_k ? warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane) : 0.f;
         if (active) {
             const float rinv = h < Hq ? rq : rk;
             uint4 *p = reinterpret_cast<uint4 *>(qkv + t * row_stride + col0);
@@ -494,14 +515,14 @@ int resident_blocks(Kern kern, KernelCache &kc, int dev, const DeviceInfo &info,
     return QKN_OK;
 }
 
-template <typename TS, int D>
-int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
-                    const float *gk, float eps, cudaStream_t stream)
+template <typename TS, int D, bool kHasK>
+int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
+                      const float *gk, float eps, cudaStream_t stream)
 {
     constexpr int U = kPerHeadRowsInFlight;
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kLPR = kNV < 32 ? kNV : 32;
-    auto kern = qkn_per_head_kernel<TS, D, U>;
+    auto kern = qkn_per_head_kernel<TS, D, U, kHasK>;
     static KernelCache kc;
     int dev = 0, per_sm = 0, rc;
     DeviceInfo info;
@@ -509,16 +530,25 @@ int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, co
     if ((rc = resident_blocks(kern, kc, dev, info, kPerHeadThreads, 0, &per_sm)) != QKN_OK)
         return rc;
     if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
-    // Qwen3 gamma is shared by every head: pass nullptr for K when Hk == 0.
-    const float *gq_eff = Hq > 0 ? gq : gk;
-    const float *gk_eff = Hk > 0 ? gk : nullptr;
     const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
     const uint64_t rows_per_block = (uint64_t)(kPerHeadThreads / kLPR) * U;
     const uint64_t need = (rows + rows_per_block - 1) / rows_per_block;
     const uint64_t cap = (uint64_t)info.sms * per_sm;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, static_cast<TS *>(qkv), row_stride,
-                      rows, (uint32_t)(Hq + Hk), (uint32_t)Hq, gq_eff, gk_eff, eps);
+    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, static_cast<TS *>(qkv), row_stride, T,
+                      (uint32_t)(Hq + Hk), (uint32_t)Hq, gq, gk, eps);
+}
+
+// Only one weight is in use when a kind of head is absent: with no key heads
+// every row is a query row, and with no query heads every row is a key row.
+template <typename TS, int D>
+int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
+                    const float *gk, float eps, cudaStream_t stream)
+{
+    if (Hq > 0 && Hk > 0)
+        return launch_per_head_k<TS, D, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps, stream);
+    const float *g = Hq > 0 ? gq : gk;
+    return launch_per_head_k<TS, D, false>(qkv, T, Hq, Hk, row_stride, g, nullptr, eps, stream);
 }
 
 // A layerwise kernel variant exists when a head splits into whole 16-byte
