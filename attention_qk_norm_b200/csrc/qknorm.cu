@@ -28,6 +28,7 @@
 // earlier in the stream always finishes first, and they allow the next
 // kernel to be scheduled as soon as all of their blocks are resident.  No
 // kernel here waits on another block, so none can hang.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -287,11 +288,16 @@ __device__ __forceinline__ float warp_rinv(const float *part, int nh, int nshard
     return rsqrtf(v / len + eps);
 }
 
-// A block of roundup32(heads * NV / VPT) threads; thread (h, l) owns vectors
-// l, l + LPH, ... of head h (LPH = NV / VPT lanes per head).  Dynamic shared
-// memory: kLayerwiseStages token stages of span = heads*D*sizeof(TS) bytes,
-// then two buffers of `heads` fp32 head partials (alternating per token).
-template <typename TS, int D, int VPT, bool kGammaRegs>
+// A token's heads are split over the CL blocks of a thread-block cluster
+// (CL = 1 for a plain launch): block c of a cluster owns heads
+// [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
+// thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
+// per head).  Dynamic shared memory per block: kLayerwiseStages stages of
+// this block's part of a token (hc*D*sizeof(TS) bytes), then two buffers of
+// `heads` fp32 head partials (alternating per token).  With CL > 1 every block
+// writes its head partials into all blocks of its cluster (distributed shared
+// memory) before the cluster barrier, so each block then holds all of them.
+template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster>
 __global__ void __launch_bounds__(1024)
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                      int nshards, const float *__restrict__ gamma_q,
@@ -307,18 +313,27 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
 
     extern __shared__ __align__(16) unsigned char smem[];
     const int heads = Hq + Hk;
-    const int span = heads * D * (int)sizeof(TS);
+    int cl = 1, crank = 0;
+    if constexpr (kCluster) {
+        cl = (int)cooperative_groups::this_cluster().num_blocks();
+        crank = (int)cooperative_groups::this_cluster().block_rank();
+    }
+    const int hc = heads / cl;           // heads of this block
+    const int h_lo = crank * hc;
+    const int span = hc * D * (int)sizeof(TS);
     float *part = reinterpret_cast<float *>(smem + (size_t)NST * span);
-    const int h = threadIdx.x / kLPH;
+    const int hl = threadIdx.x / kLPH;   // head within this block
+    const int h = h_lo + hl;
     const int l = threadIdx.x % kLPH;
-    const bool active = h < heads;
+    const bool active = hl < hc;
     const int lane = threadIdx.x % 32;
     // Heads of this warp's threads; a warp computes only the inverse RMS of
     // the vectors it holds (warp-uniform, so whole warps shuffle together).
-    const int warp_first_head = (threadIdx.x & ~31) / kLPH;
-    const int warp_last_head = (threadIdx.x | 31) / kLPH;
+    const int warp_first_head = h_lo + (threadIdx.x & ~31) / kLPH;
+    const int warp_last_head = h_lo + (threadIdx.x | 31) / kLPH;
     const bool need_q = warp_first_head < Hq;
     const bool need_k = Hk > 0 && warp_last_head >= Hq;
+    const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
 
     pdl_wait_then_release();
     const float *gb = !active ? gamma_q
@@ -335,26 +350,26 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
             for (int e = 0; e < kVec; ++e) g[v * kVec + e] = t4[e];
         }
     }
-    const int64_t col0 = (int64_t)h * D;
+    const int64_t col0 = (int64_t)h * D;              // in the token row
+    const size_t scol0 = (size_t)hl * D * sizeof(TS);  // in a stage
     // Each thread copies, and later reads, only its own vectors of a stage.
     auto fetch = [&](int64_t tok, int st) {
         if (active && tok < T) {
             const uint4 *src = reinterpret_cast<const uint4 *>(qkv + tok * row_stride + col0);
-            unsigned char *dst = smem + (size_t)st * span + col0 * sizeof(TS);
+            unsigned char *dst = smem + (size_t)st * span + scol0;
 #pragma unroll
             for (int v = 0; v < VPT; ++v) cp_async16(dst + (l + v * kLPH) * 16, src + l + v * kLPH);
         }
         cp_async_commit();
     };
 #pragma unroll
-    for (int i = 0; i < NST - 1; ++i) fetch(blockIdx.x + (int64_t)i * gridDim.x, i);
+    for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
     int st = 0, pb = 0;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    for (int64_t t = first; t < T; t += stride) {
         // Refill the stage this thread finished with on the previous token.
-        fetch(t + (int64_t)(NST - 1) * gridDim.x, (st + NST - 1) % NST);
+        fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
         cp_async_wait<NST - 1>();
-        const uint4 *sp =
-            reinterpret_cast<const uint4 *>(smem + (size_t)st * span + col0 * sizeof(TS));
+        const uint4 *sp = reinterpret_cast<const uint4 *>(smem + (size_t)st * span + scol0);
         float s = 0.f;
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
@@ -366,10 +381,17 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         s = group_sum<kLPH>(s);
         // Partials alternate between two buffers: a warp still reading this
         // token's buffer cannot meet a write of the next token's, which only
-        // starts after the next barrier.
+        // starts after the next barrier (of the block, or of the cluster).
         float *pp = part + pb * heads;
-        if (active && l == 0) pp[h] = s;
-        __syncthreads();
+        if constexpr (kCluster) {
+            cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+            if (active && l == 0)
+                for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(pp + h, r) = s;
+            cluster.sync();
+        } else {
+            if (active && l == 0) pp[h] = s;
+            __syncthreads();
+        }
         const float rq = need_q ? warp_rinv(pp, Hq, nshards, len_q, eps, lane) : 0.f;
         const float rk = need_k ? warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane) : 0.f;
         if (active) {
@@ -435,21 +457,26 @@ int device_info(int *dev_out, DeviceInfo *info)
 }
 
 // Launch with programmatic stream serialization allowed (see the kernels'
-// griddepcontrol.wait), then report the launch status.
+// griddepcontrol.wait) and, when cluster > 1, as clusters of `cluster`
+// blocks along x; then report the launch status.
 template <typename... Params, typename... Args>
 int launch_pdl(void (*kern)(Params...), unsigned grid, unsigned threads, size_t smem,
-               cudaStream_t stream, Args... args)
+               cudaStream_t stream, unsigned cluster, Args... args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = cluster > 1 ? 2 : 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
     if (e == cudaSuccess) e = cudaGetLastError();
     return e == cudaSuccess ? QKN_OK : cuda_fail(e);
@@ -535,7 +562,7 @@ int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, 
     const uint64_t need = (rows + rows_per_block - 1) / rows_per_block;
     const uint64_t cap = (uint64_t)info.sms * per_sm;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, static_cast<TS *>(qkv), row_stride, T,
+    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, 1u, static_cast<TS *>(qkv), row_stride, T,
                       (uint32_t)(Hq + Hk), (uint32_t)Hq, gq, gk, eps);
 }
 
@@ -567,45 +594,88 @@ constexpr bool layerwise_gamma_regs()
     return VPT * Storage<TS>::kVec <= 32;
 }
 
-template <typename TS, int D, int VPT>
+template <typename TS, int D, int VPT, bool kCluster>
 int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
                          const float *gq, const float *gk, float eps, int nshards, int threads,
-                         cudaStream_t stream)
+                         int cluster, cudaStream_t stream)
 {
-    auto kern = qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>()>;
+    auto kern = qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>(), kCluster>;
     static KernelCache kc;
     const int heads = Hq + Hk;
-    const size_t span = (size_t)heads * D * sizeof(TS);
+    const size_t span = (size_t)(heads / cluster) * D * sizeof(TS);
     const size_t smem = kLayerwiseStages * span + (size_t)2 * heads * sizeof(float);
-    int dev = 0, per_sm = 0, rc;
+    int dev = 0, rc;
     DeviceInfo info;
     if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
     if (smem > (size_t)info.smem_optin) return QKN_ERR_UNSUPPORTED;
-    if ((rc = resident_blocks(kern, kc, dev, info, threads, smem, &per_sm)) != QKN_OK) return rc;
-    if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
-    const int64_t cap = (int64_t)info.sms * per_sm;
-    const unsigned grid = (unsigned)(T < cap ? T : cap);
+    int64_t cap = 0;  // co-resident clusters (of `cluster` blocks) on the device
+    if (kCluster) {
+        if (smem > 48 * 1024 && !(kc.smem_ready.load(std::memory_order_acquire) & (1ull << dev))) {
+            const cudaError_t e = cudaFuncSetAttribute(
+                kern, cudaFuncAttributeMaxDynamicSharedMemorySize, info.smem_optin);
+            if (e != cudaSuccess) return cuda_fail(e);
+            kc.smem_ready.fetch_or(1ull << dev, std::memory_order_acq_rel);
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)cluster);
+        cfg.blockDim = dim3((unsigned)threads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)cluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return cuda_fail(e);
+        cap = n;
+    } else {
+        int per_sm = 0;
+        if ((rc = resident_blocks(kern, kc, dev, info, threads, smem, &per_sm)) != QKN_OK) return rc;
+        cap = (int64_t)info.sms * per_sm;
+    }
+    if (cap < 1) return QKN_ERR_UNSUPPORTED;
+    const int64_t clusters = T < cap ? T : cap;
     const float len_q = (float)((int64_t)Hq * D);  // exact: spans are < 2^24 elements
     const float len_k = (float)((int64_t)Hk * D);
-    return launch_pdl(kern, grid, threads, smem, stream, static_cast<TS *>(qkv), row_stride, T,
-                      Hq, Hk, nshards, gq, gk, eps, len_q, len_k);
+    return launch_pdl(kern, (unsigned)(clusters * cluster), threads, smem, stream,
+                      (unsigned)cluster, static_cast<TS *>(qkv), row_stride, T, Hq, Hk, nshards,
+                      gq, gk, eps, len_q, len_k);
 }
 
-// Vectors per thread: the fewest that keep a token's block within 256
-// threads, else within 1024.
+// Launch shape.  First choice: the smallest cluster (1, 2, 4 or 8 blocks,
+// dividing the head count) and the fewest vectors per thread that keep gamma
+// in registers and the block within 256 threads.  Otherwise one block per
+// token, the fewest vectors per thread within 256 threads, else 1024, with
+// gamma read through L1 where it does not fit registers.
 constexpr int kLayerwiseTargetThreads = 256;
+constexpr int kMaxCluster = 8;
 
 template <typename TS, int D>
 int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                      const float *gk, float eps, int nshards, cudaStream_t stream)
 {
     constexpr int kNV = D / Storage<TS>::kVec;
+    constexpr int kVec = Storage<TS>::kVec;
     const int64_t heads = Hq + Hk;
-    int chosen = 0;
+    int chosen = 0, cluster = 1;
+    for (int cl = 1; cl <= kMaxCluster && chosen == 0; cl *= 2) {
+        if (heads % cl != 0) continue;
+        for (int vpt = 1; vpt <= kNV && vpt * kVec <= 32; vpt *= 2) {
+            if (kNV % vpt != 0 || kNV / vpt > 32) continue;  // mirrors layerwise_vpt_ok
+            if (((heads / cl * (kNV / vpt) + 31) / 32) * 32 <= kLayerwiseTargetThreads) {
+                chosen = vpt;
+                cluster = cl;
+                break;
+            }
+        }
+    }
     for (int pass = 0; pass < 2 && chosen == 0; ++pass) {
         const int64_t limit = pass == 0 ? kLayerwiseTargetThreads : 1024;
         for (int vpt = 1; vpt <= kNV; vpt *= 2) {
-            if (kNV % vpt != 0 || kNV / vpt > 32) continue;  // mirrors layerwise_vpt_ok
+            if (kNV % vpt != 0 || kNV / vpt > 32) continue;
             if (((heads * (kNV / vpt) + 31) / 32) * 32 <= limit) {
                 chosen = vpt;
                 break;
@@ -613,12 +683,19 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
         }
     }
     if (chosen == 0) return QKN_ERR_UNSUPPORTED;
-    const int threads = (int)(((heads * (kNV / chosen) + 31) / 32) * 32);
+    const int threads = (int)(((heads / cluster * (kNV / chosen)) + 31) / 32 * 32);
 #define QKN_LW_CASE(V)                                                                         \
     case V:                                                                                    \
-        if constexpr (layerwise_vpt_ok<TS, D, V>())                                            \
-            return launch_layerwise_vpt<TS, D, V>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,     \
-                                                  nshards, threads, stream);                   \
+        if constexpr (layerwise_vpt_ok<TS, D, V>()) {                                          \
+            if constexpr (layerwise_gamma_regs<TS, V>()) {                                     \
+                if (cluster > 1)                                                               \
+                    return launch_layerwise_vpt<TS, D, V, true>(qkv, T, Hq, Hk, row_stride,    \
+                                                                gq, gk, eps, nshards, threads, \
+                                                                cluster, stream);              \
+            }                                                                                  \
+            return launch_layerwise_vpt<TS, D, V, false>(qkv, T, Hq, Hk, row_stride, gq, gk,   \
+                                                         eps, nshards, threads, 1, stream);    \
+        }                                                                                      \
         break;
     switch (chosen) {
         QKN_LW_CASE(1)

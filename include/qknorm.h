@@ -98,11 +98,12 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
  * length.  nshards is 1, 2, 4 or 8 and must divide both Hq and Hk.  All
  * shards run inside one kernel on one GPU; there is no cross-GPU traffic.
  * The reduction is a fixed tree whose subtrees are the shards, so the output
- * is bit-identical for every valid nshards.  One thread block works on one
- * token at a time and keeps two tokens staged in shared memory, so the Q+K
- * span must satisfy 2 * (Hq + Hk) * D * sizeof(element) + 8 * (Hq + Hk)
- * <= the device's opt-in shared memory per block (227 KiB on B200), else
- * QKN_ERR_UNSUPPORTED.
+ * is bit-identical for every valid nshards.  A token's heads are split over
+ * a thread-block cluster of 1, 2, 4 or 8 blocks (C, which must divide
+ * Hq + Hk); each block keeps two tokens' worth of its heads staged in shared
+ * memory, so 2 * (Hq + Hk) / C * D * sizeof(element) + 8 * (Hq + Hk) bytes
+ * must fit the device's opt-in shared memory per block (227 KiB on B200) for
+ * the cluster size chosen, else QKN_ERR_UNSUPPORTED.
  */
 int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
                      const float *gamma_q, const float *gamma_k, float eps, int nshards,

@@ -174,6 +174,22 @@ def test_layerwise_head_counts(Hq, Hk, ns):
         assert np.array_equal(o, outs[0])
 
 
+@pytest.mark.parametrize("dtype", (synth.BF16, synth.FP32))
+@pytest.mark.parametrize("D", synth.STRESS_D)
+@pytest.mark.parametrize("Hq,Hk,ns", [(64, 8, (1, 8)), (32, 4, (1, 4)), (30, 5, (1, 5))])
+def test_layerwise_wide_tokens(dtype, D, Hq, Hk, ns):
+    """Wide tokens: heads split over a thread-block cluster (72 or 36 heads),
+    or one block with gamma read through L1 (35 heads: no cluster size
+    divides the head count)."""
+    ns = tuple(n for n in ns if n in (1, 2, 4, 8))
+    c = synth.make_case(45, Hq, Hk, D, dtype=dtype, seed=Hq + D, layerwise=True, scale="stress",
+                        zero_frac=0.05, outlier_frac=0.05)
+    outs = [full_parity(c, "layerwise", n, what="wide %s D=%d n=%d" % (dtype, D, n))[0]
+            for n in ns]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
 def test_zero_eps_on_nonzero_rows():
     c = synth.make_case(64, 4, 2, 128, seed=21, eps=0.0)
     full_parity(c, "per_head", what="eps=0")
@@ -205,11 +221,12 @@ def test_errors_leave_buffer_untouched():
     with pytest.raises(qkn.QKNormError) as e:
         qkn.qknorm_layerwise(full, 16, 2, 128, gq, gk, 1e-6, nshards=4)
     assert e.value.status == -4
-    # 136 fp32 heads of 256: two staged tokens need 272 KiB of shared memory
-    wide = torch.zeros((1, (128 + 16) * 256), dtype=torch.float32, device="cuda")
-    g = torch.ones(128 * 256, device="cuda")
+    # 137 fp32 heads of 256: an odd head count rules out a cluster split, and
+    # two staged tokens in one block would need 274 KiB of shared memory
+    wide = torch.zeros((1, (129 + 16) * 256), dtype=torch.float32, device="cuda")
+    g = torch.ones(129 * 256, device="cuda")
     with pytest.raises(qkn.QKNormError) as e:
-        qkn.qknorm_layerwise(wide, 128, 8, 256, g, g, 1e-6)
+        qkn.qknorm_layerwise(wide, 129, 8, 256, g, g, 1e-6)
     assert e.value.status == -5
     torch.cuda.synchronize()
     assert torch.equal(full.view(torch.int16), before.view(torch.int16))
