@@ -533,6 +533,9 @@ PROFILE_CASES = {
                 scale="lognormal", seed=1002),
     "layerwise": dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
                       nshards=8, seed=1003),
+    "layerwise_wide": dict(kind="layerwise", T=8192, Hq=64, Hk=8, D=128, dtype="bf16", eps=1e-6,
+                           nshards=8, scale="stress", zero_frac=0.01, outlier_frac=0.01,
+                           seed=1004),
 }
 
 
