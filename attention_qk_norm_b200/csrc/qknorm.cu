@@ -364,6 +364,11 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     };
 #pragma unroll
     for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
+    // Distributed shared memory may only be touched once every block of the
+    // cluster is running: meet once before the first remote write.  (The last
+    // remote write of the loop precedes its final cluster barrier, so no block
+    // exits while another may still write into it.)
+    if constexpr (kCluster) cooperative_groups::this_cluster().sync();
     int st = 0, pb = 0;
     for (int64_t t = first; t < T; t += stride) {
         // Refill the stage this thread finished with on the previous token.
