@@ -8,6 +8,8 @@ package, or ``synth`` alone, needs neither the library nor a GPU.
 """
 from ._binding import (  # noqa: F401
     QKN_BF16,
+    QKN_FP8_E4M3,
+    QKN_FP16,
     QKN_FP32,
     QKNormError,
     load_library,

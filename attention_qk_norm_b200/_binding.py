@@ -13,7 +13,7 @@ import threading
 
 from .buildlib import LIB_PATH
 
-QKN_BF16, QKN_FP32 = 0, 1
+QKN_BF16, QKN_FP32, QKN_FP16, QKN_FP8_E4M3 = 0, 1, 2, 3
 STATUS = {
     0: "QKN_OK", -1: "QKN_ERR_NULL", -2: "QKN_ERR_SHAPE", -3: "QKN_ERR_ALIGN",
     -4: "QKN_ERR_NSHARDS", -5: "QKN_ERR_UNSUPPORTED", -6: "QKN_ERR_CUDA", -7: "QKN_ERR_EPS",
@@ -74,11 +74,12 @@ def _check(fn: str, rc: int) -> None:
 def _dtype_code(t) -> int:
     import torch
 
-    if t.dtype == torch.bfloat16:
-        return QKN_BF16
-    if t.dtype == torch.float32:
-        return QKN_FP32
-    raise TypeError("qkv must be bfloat16 or float32, got %s" % t.dtype)
+    codes = {torch.bfloat16: QKN_BF16, torch.float32: QKN_FP32, torch.float16: QKN_FP16,
+             torch.float8_e4m3fn: QKN_FP8_E4M3}
+    if t.dtype not in codes:
+        raise TypeError("qkv must be bfloat16, float32, float16 or float8_e4m3fn, got %s"
+                        % t.dtype)
+    return codes[t.dtype]
 
 
 def _rows(qkv, row_stride):

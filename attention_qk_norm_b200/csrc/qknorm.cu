@@ -30,6 +30,8 @@
 // kernel here waits on another block, so none can hang.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <math.h>
@@ -89,6 +91,67 @@ struct Storage<float> {
     }
 };
 
+template <>
+struct Storage<__half> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            f[2 * i] = p.x;
+            f[2 * i + 1] = p.y;
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[8])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2 p = __floats2half2_rn(f[2 * i], f[2 * i + 1]);  // round to nearest even
+            w[i] = *reinterpret_cast<uint32_t *>(&p);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+// FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per vector.
+// Decoded exactly through fp16; encoded round-to-nearest-even, saturating to
+// +-448.  The lower byte of each pair is the earlier element.
+template <>
+struct Storage<__nv_fp8_e4m3> {
+    static constexpr int kVec = 16;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[16])
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
+                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&r));
+                f[4 * i + 2 * j] = p.x;
+                f[4 * i + 2 * j + 1] = p.y;
+            }
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[16])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i], f[4 * i + 1]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i + 2], f[4 * i + 3]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            w[i] = lo | (hi << 16);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
 // Streaming (evict-first) 16-byte accesses: each element is touched once.
 __device__ __forceinline__ uint4 load_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void store_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
@@ -144,14 +207,18 @@ __device__ __forceinline__ void cp_async_wait()
 // ---------------------------------------------------------------- per-head --
 constexpr int kPerHeadThreads = 256;
 constexpr int kPerHeadRowsInFlight = 2;
-// Resident 256-thread blocks per SM that the register budget must allow:
-// six (40 registers) for the single-weight loop with one vector per lane and
-// row, five (48) with both weights, four (64) with two vectors per lane.
-// Each fits without spilling.
+// Resident 256-thread blocks per SM that the register budget must allow, by
+// elements a lane holds per row: six (40 registers) for the single-weight
+// loop with 8 elements, five (48) with both weights; four (64) and three (80)
+// for FP8's 16 elements; four for fp32 D=256 (two vectors per lane).  Each
+// fits without spilling.
 template <typename TS, int D, bool kHasK>
 constexpr int per_head_min_blocks()
 {
-    return D / Storage<TS>::kVec > 32 ? 4 : (kHasK ? 5 : 6);
+    constexpr int kNV = D / Storage<TS>::kVec;
+    constexpr int kVPL = kNV > 32 ? kNV / 32 : 1;
+    constexpr int kEPL = kVPL * Storage<TS>::kVec;
+    return kVPL > 1 ? 4 : (kEPL > 8 ? (kHasK ? 3 : 4) : (kHasK ? 5 : 6));
 }
 
 // Rows are visited with a grid stride: thread group g takes rows g, g + G,
@@ -489,7 +556,16 @@ int launch_pdl(void (*kern)(Params...), unsigned grid, unsigned threads, size_t 
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-int elem_size(int dtype) { return dtype == QKN_BF16 ? 2 : (dtype == QKN_FP32 ? 4 : 0); }
+int elem_size(int dtype)
+{
+    switch (dtype) {
+    case QKN_BF16: return 2;
+    case QKN_FP32: return 4;
+    case QKN_FP16: return 2;
+    case QKN_FP8_E4M3: return 1;
+    default: return 0;
+    }
+}
 
 // Checks shared by both entry points.  Order: dtype, shape, eps, T == 0,
 // pointers, alignment.
@@ -717,6 +793,34 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
     return QKN_ERR_UNSUPPORTED;
 }
 
+// Storage type and head_dim as template arguments of F::run.
+template <typename F, typename... Args>
+int dispatch(int dtype, int D, Args... args)
+{
+#define QKN_BY_D(TS)                                                                           \
+    switch (D) {                                                                               \
+    case 64: return F::template run<TS, 64>(args...);                                          \
+    case 128: return F::template run<TS, 128>(args...);                                        \
+    default: return F::template run<TS, 256>(args...);                                         \
+    }
+    switch (dtype) {
+    case QKN_BF16: QKN_BY_D(__nv_bfloat16)
+    case QKN_FP32: QKN_BY_D(float)
+    case QKN_FP16: QKN_BY_D(__half)
+    default: QKN_BY_D(__nv_fp8_e4m3)
+    }
+#undef QKN_BY_D
+}
+
+struct PerHead {
+    template <typename TS, int D, typename... A>
+    static int run(A... a) { return launch_per_head<TS, D>(a...); }
+};
+struct Layerwise {
+    template <typename TS, int D, typename... A>
+    static int run(A... a) { return launch_layerwise<TS, D>(a...); }
+};
+
 }  // namespace
 
 extern "C" {
@@ -727,19 +831,8 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
     bool done = false;
     const int rc = validate(qkv, dtype, T, Hq, Hk, D, row_stride, gamma_q, gamma_k, eps, &done);
     if (rc != QKN_OK || done) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == QKN_BF16) {
-        switch (D) {
-        case 64: return launch_per_head<__nv_bfloat16, 64>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-        case 128: return launch_per_head<__nv_bfloat16, 128>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-        default: return launch_per_head<__nv_bfloat16, 256>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-        }
-    }
-    switch (D) {
-    case 64: return launch_per_head<float, 64>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-    case 128: return launch_per_head<float, 128>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-    default: return launch_per_head<float, 256>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, s);
-    }
+    return dispatch<PerHead>(dtype, D, qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps,
+                             static_cast<cudaStream_t>(stream));
 }
 
 int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
@@ -752,19 +845,8 @@ int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int
     if (nshards != 1 && nshards != 2 && nshards != 4 && nshards != 8) return QKN_ERR_NSHARDS;
     if (Hq % nshards != 0 || Hk % nshards != 0) return QKN_ERR_NSHARDS;
     if (done) return QKN_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == QKN_BF16) {
-        switch (D) {
-        case 64: return launch_layerwise<__nv_bfloat16, 64>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-        case 128: return launch_layerwise<__nv_bfloat16, 128>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-        default: return launch_layerwise<__nv_bfloat16, 256>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-        }
-    }
-    switch (D) {
-    case 64: return launch_layerwise<float, 64>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-    case 128: return launch_layerwise<float, 128>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-    default: return launch_layerwise<float, 256>(qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps, nshards, s);
-    }
+    return dispatch<Layerwise>(dtype, D, qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps,
+                               nshards, static_cast<cudaStream_t>(stream));
 }
 
 const char *qknorm_status_string(int status)
@@ -784,6 +866,6 @@ const char *qknorm_status_string(int status)
 
 int qknorm_last_cuda_error(void) { return g_last_cuda_error; }
 
-int qknorm_version(void) { return 100; }
+int qknorm_version(void) { return 101; }
 
 }  // extern "C"

@@ -2,7 +2,10 @@
 
 This module holds no QK-Norm arithmetic: it only draws random activations
 and weights with the shapes and value distributions of the workloads, and
-stores them in bf16 (round-to-nearest-even from float32) or fp32.  The
+stores them in bf16 or fp16 (round-to-nearest-even from float32), FP8 E4M3
+(round-to-nearest-even; magnitudes beyond its largest finite value, 448,
+become 448, which also turns the stress recipe's 1e4 outliers into 448), or
+fp32.  The
 oracle (``oracle/``) and the CUDA path both consume what it produces; it
 imports neither of them.
 
@@ -39,6 +42,9 @@ import numpy as np
 
 BF16 = "bf16"
 FP32 = "fp32"
+FP16 = "fp16"
+FP8 = "fp8_e4m3"
+E4M3_MAX = 448.0
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -51,11 +57,54 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return ((b + bias) >> np.uint32(16)).astype(np.uint16)
 
 
+def f32_to_fp16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to IEEE binary16 (nearest, ties to even); uint16 bits."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def _e4m3_magnitudes() -> np.ndarray:
+    """Values of the non-negative finite FP8 E4M3 codes 0..126, increasing:
+    4 exponent bits (bias 7) and 3 mantissa bits, subnormals at exponent 0;
+    code 127 is NaN, so 126 (448) is the largest finite value."""
+    codes = np.arange(127)
+    e, m = codes >> 3, codes & 7
+    return np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+
+
+_E4M3 = _e4m3_magnitudes()
+
+
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round to FP8 E4M3 (nearest, ties to the even code); magnitudes beyond
+    448 become 448.  Returns uint8 codes (sign in bit 7)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3, a, side="left"), 0, 126)
+    lo = np.clip(hi - 1, 0, 126)
+    d_lo, d_hi = a - _E4M3[lo], _E4M3[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return code | (np.signbit(x).astype(np.uint8) << np.uint8(7))
+
+
+def store(x: np.ndarray, dtype: str) -> np.ndarray:
+    """float32 values in the storage format of ``dtype`` (bits or values)."""
+    if dtype == BF16:
+        return f32_to_bf16_bits(x)
+    if dtype == FP16:
+        return f32_to_fp16_bits(x)
+    if dtype == FP8:
+        return f32_to_e4m3_bits(x)
+    if dtype == FP32:
+        return np.ascontiguousarray(x, dtype=np.float32)
+    raise ValueError("unknown dtype %r" % (dtype,))
+
+
 @dataclasses.dataclass
 class Case:
     """One synthetic QK-Norm input: fused buffer, weights and shape."""
 
-    qkv: np.ndarray  # [T, row_stride]; uint16 bf16 bits or float32
+    qkv: np.ndarray  # [T, row_stride]; uint16 bf16/fp16 bits, uint8 e4m3 codes, or float32
     gamma_q: np.ndarray  # float32
     gamma_k: Optional[np.ndarray]  # float32 or None when Hk == 0
     T: int
@@ -101,7 +150,7 @@ def make_case(T, Hq, Hk, D, *, dtype=BF16, seed=0, row_stride=None, layerwise=Fa
     lq, lk = (Hq * D, Hk * D) if layerwise else (D, D)
     gamma_q = (1.0 + 0.1 * rng.standard_normal(lq)).astype(np.float32)
     gamma_k = (1.0 + 0.1 * rng.standard_normal(lk)).astype(np.float32) if Hk > 0 else None
-    qkv = f32_to_bf16_bits(x) if dtype == BF16 else x
+    qkv = store(x, dtype)
     return Case(qkv, gamma_q, gamma_k, T, Hq, Hk, D, stride, dtype, eps, layerwise)
 
 
@@ -116,7 +165,8 @@ def make_case_torch(T, Hq, Hk, D, *, device, dtype=BF16, seed=0, row_stride=None
         raise ValueError("row_stride must be >= (Hq + 2*Hk) * D")
     g = torch.Generator(device=device)
     g.manual_seed(seed)
-    tdt = torch.bfloat16 if dtype == BF16 else torch.float32
+    tdt = {BF16: torch.bfloat16, FP32: torch.float32, FP16: torch.float16,
+           FP8: torch.float8_e4m3fn}[dtype]
     qkv = torch.empty((T, stride), dtype=tdt, device=device)
     # Draw in float32 slabs so the temporary stays small for multi-GB buffers.
     slab = max(1, (1 << 26) // max(1, stride))
@@ -131,6 +181,8 @@ def make_case_torch(T, Hq, Hk, D, *, device, dtype=BF16, seed=0, row_stride=None
             x *= s.clamp_(1e-3, 1e3)
         elif scale is not None:
             raise ValueError("unknown scale recipe %r" % (scale,))
+        if dtype == FP8:
+            x.clamp_(-E4M3_MAX, E4M3_MAX)  # E4M3 has no infinities
         qkv[t0:t1] = x.to(tdt)
         del x
     qk = (Hq + Hk) * D
@@ -141,7 +193,8 @@ def make_case_torch(T, Hq, Hk, D, *, device, dtype=BF16, seed=0, row_stride=None
         qkv[zero_rows, :qk] = 0
         cols = torch.randint(0, qk, (out_rows.numel(),), generator=g, device=device)
         signs = torch.randint(0, 2, (out_rows.numel(),), generator=g, device=device) * 2 - 1
-        qkv[out_rows, cols] = (signs.float() * 1e4).to(tdt)
+        big = E4M3_MAX if dtype == FP8 else 1e4
+        qkv[out_rows, cols] = (signs.float() * big).to(tdt)
     lq, lk = (Hq * D, Hk * D) if layerwise else (D, D)
     gamma_q = 1.0 + 0.1 * torch.randn(lq, generator=g, device=device, dtype=torch.float32)
     gamma_k = (1.0 + 0.1 * torch.randn(lk, generator=g, device=device, dtype=torch.float32)

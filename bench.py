@@ -56,9 +56,12 @@ HEADLINE_NAME = ("per-head QK-Norm, head_dim 128, 48 heads, T=4096 tokens, bf16,
 
 
 # ---------------------------------------------------------------- helpers --
+ELEM_BYTES = {"bf16": 2, "fp16": 2, "fp32": 4, "fp8_e4m3": 1}
+
+
 def workload_bytes(w) -> int:
     """Algorithmic bytes of one call: read + write of Q and K once, gamma once."""
-    es = 2 if w["dtype"] == "bf16" else 4
+    es = ELEM_BYTES[w["dtype"]]
     qk = (w["Hq"] + w["Hk"]) * w["D"]
     if w["kind"] == "per_head":
         gamma = w["D"] * 4 * ((w["Hq"] > 0) + (w["Hk"] > 0))
@@ -294,6 +297,12 @@ def extra_workloads():
             out.append(("layerwise n=%d" % n, dict(kind="layerwise", T=T, Hq=32, Hk=8, D=128,
                                                     dtype="bf16", eps=1e-6, nshards=n,
                                                     seed=2300 + T)))
+    for dt in (synth.FP16, synth.FP8):
+        out.append(("gqa fused 32q/8kv %s" % dt, dict(kind="per_head", T=16384, Hq=32, Hk=8,
+                                                      D=128, dtype=dt, eps=1e-6, nshards=1,
+                                                      scale="lognormal", seed=2500)))
+        out.append(("layerwise n=8 %s" % dt, dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128,
+                                                  dtype=dt, eps=1e-6, nshards=8, seed=2600)))
     for dt in synth.STRESS_DTYPES:
         for D in synth.STRESS_D:
             for kind in ("per_head", "layerwise"):

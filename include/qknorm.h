@@ -18,11 +18,13 @@
  * Arithmetic: elements are widened to fp32, sums of squares accumulate in
  * fp32, the inverse RMS is 1/sqrt(S/L + eps) in fp32 (L = normalised length,
  * eps inside the square root), and each output x * rinv * gamma is rounded
- * once to the storage type (round to nearest even for bf16).
+ * once to the storage type: round to nearest even for bf16 and fp16, and for
+ * FP8 E4M3 round to nearest even saturating to +-448.
  *
  * Common arguments
  *   qkv         device pointer to the fused buffer; 16-byte aligned.
- *   dtype       QKN_BF16 or QKN_FP32 (storage type of qkv).
+ *   dtype       QKN_BF16, QKN_FP32, QKN_FP16 or QKN_FP8_E4M3 (storage type
+ *               of qkv).
  *   T           number of tokens (rows), >= 0; T == 0 returns QKN_OK and
  *               launches nothing (qkv may then be NULL).
  *   Hq, Hk      query / key head counts, >= 0, Hq + Hk >= 1.
@@ -56,7 +58,12 @@
 extern "C" {
 #endif
 
-typedef enum { QKN_BF16 = 0, QKN_FP32 = 1 } qkn_dtype;
+typedef enum {
+    QKN_BF16 = 0,     /* bfloat16                                            */
+    QKN_FP32 = 1,     /* IEEE binary32                                       */
+    QKN_FP16 = 2,     /* IEEE binary16                                       */
+    QKN_FP8_E4M3 = 3  /* FP8 E4M3 (bias 7, no infinities, max finite 448)    */
+} qkn_dtype;
 
 typedef enum {
     QKN_OK = 0,
@@ -115,7 +122,7 @@ const char *qknorm_status_string(int status);
 /* cudaError_t of the calling thread's last QKN_ERR_CUDA (0 if none). */
 int qknorm_last_cuda_error(void);
 
-/* ABI version: 100 * major + minor. */
+/* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3). */
 int qknorm_version(void);
 
 #ifdef __cplusplus

@@ -19,7 +19,9 @@ Definitions followed (the header of ``qknorm_oracle.c`` states them in full):
   projection" lesson, GQA section and tensor-parallel follow-up.
 
 Inputs are widened exactly to float64 here: bf16 bit patterns (uint16) are
-shifted into the high half of a float32, float32 values are cast.  The
+shifted into the high half of a float32, fp16 bit patterns are read as IEEE
+binary16, FP8 E4M3 codes are decoded from the format's definition, float32
+values are cast.  The
 oracle is pinned by closed forms and invariants (``tests/pins.py``).
 """
 from __future__ import annotations
@@ -39,6 +41,28 @@ _default = None
 
 BF16 = "bf16"
 FP32 = "fp32"
+FP16 = "fp16"
+FP8 = "fp8_e4m3"
+
+
+def _e4m3_table() -> np.ndarray:
+    """float64 value of each of the 256 FP8 E4M3 codes: sign bit 7, exponent
+    bits 6..3 with bias 7, mantissa bits 2..0; exponent 0 is subnormal
+    (m * 2^-9); 0x7f and 0xff are NaN (the format has no infinities)."""
+    out = np.empty(256)
+    for c in range(256):
+        sign = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 0xF, c & 0x7
+        if e == 0xF and m == 0x7:
+            out[c] = np.nan
+        elif e == 0:
+            out[c] = sign * m * 2.0 ** -9
+        else:
+            out[c] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return out
+
+
+_E4M3 = _e4m3_table()
 
 
 def compile_source(src: str, out: str) -> str:
@@ -59,13 +83,18 @@ def build(force: bool = False) -> str:
 
 
 def widen(x: np.ndarray, dtype: str) -> np.ndarray:
-    """Exact float64 value of stored elements (bf16 bits as uint16, or fp32)."""
+    """Exact float64 value of stored elements: bf16 / fp16 bits as uint16, FP8
+    E4M3 codes as uint8, or fp32 values."""
     if dtype == BF16:
         bits = np.ascontiguousarray(x, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
         return bits.view(np.float32).astype(np.float64)
     if dtype == FP32:
         return np.ascontiguousarray(x, dtype=np.float32).astype(np.float64)
-    raise ValueError("dtype must be 'bf16' or 'fp32'")
+    if dtype == FP16:
+        return np.ascontiguousarray(x, dtype=np.uint16).view(np.float16).astype(np.float64)
+    if dtype == FP8:
+        return _E4M3[np.ascontiguousarray(x, dtype=np.uint8)]
+    raise ValueError("dtype must be 'bf16', 'fp32', 'fp16' or 'fp8_e4m3'")
 
 
 def _dptr(a: np.ndarray):

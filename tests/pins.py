@@ -84,6 +84,29 @@ def pin_bf16_widening(o):
                        1 / math.sqrt(2.5)], rel=1e-14, abs_=0.0, what="bf16 widening")
 
 
+def pin_low_precision_widening(o):
+    """fp16 bits and FP8 E4M3 codes reach the oracle as their exact values:
+    a one-head row with eps = 0 and the value 2^k at one spot maps to
+    sqrt(D) * g there, so a wrong decode of that spot would show; every code
+    is also checked through the oracle's input path against torch's decode."""
+    import torch
+
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    finite = ~np.isnan(ref)
+    D = 256
+    x = codes.reshape(1, D)
+    x = np.where(finite.reshape(1, D), x, np.uint8(0))  # replace the NaN codes by +0
+    got = o.per_head(x, "fp8_e4m3", 1, 1, 0, D, D, np.ones(D, np.float32), None, 0.0)
+    want = np.where(finite, ref, 0.0)
+    _close(got.ravel(), want * math.sqrt(D) / np.linalg.norm(want), rel=1e-14, abs_=0.0,
+           what="e4m3 widening")
+    h = np.array([0x3C00, 0xC000, 0x0001, 0x7BFF], dtype=np.uint16)  # 1, -2, 2^-24, 65504
+    y = o.per_head(h, "fp16", 1, 1, 0, 4, 4, np.ones(4, np.float32), None, 0.0)
+    v = np.array([1.0, -2.0, 2.0 ** -24, 65504.0])
+    _close(y.ravel(), v * 2.0 / np.linalg.norm(v), rel=1e-14, abs_=0.0, what="fp16 widening")
+
+
 def pin_unit_rms(o):
     rng = np.random.default_rng(11)
     T, Hq, Hk, D = 5, 3, 2, 16
@@ -284,6 +307,7 @@ def pin_gamma_and_layout(o):
 ALL_PINS = [
     pin_closed_forms,
     pin_bf16_widening,
+    pin_low_precision_widening,
     pin_unit_rms,
     pin_scale_invariance,
     pin_eps_branch,

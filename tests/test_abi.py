@@ -17,7 +17,7 @@ from attention_qk_norm_b200 import buildlib as qbuild
 
 HEADER = os.path.join(qbuild.INCLUDE, "qknorm.h")
 OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS = 0, -1, -2, -3, -4, -5, -6, -7
-BF16, FP32 = 0, 1
+BF16, FP32, FP16, FP8 = 0, 1, 2, 3
 # Fake, never-dereferenced addresses: validation rejects before any access.
 P, G1, G2 = 0x100000, 0x200000, 0x300000
 
@@ -47,7 +47,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.qknorm_version() == 100
+    assert lib.qknorm_version() == 101
     for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS):
         s = lib.qknorm_status_string(code).decode()
         assert s and s != "unknown status"
@@ -68,7 +68,8 @@ def lw(lib, qkv=P, dtype=BF16, T=4, Hq=32, Hk=8, D=128, stride=None, gq=G1, gk=G
 
 @pytest.mark.parametrize("fn", [ph, lw])
 def test_validation(lib, fn):
-    assert fn(lib, dtype=2) == UNSUP
+    assert fn(lib, dtype=4) == UNSUP
+    assert fn(lib, dtype=-1) == UNSUP
     assert fn(lib, D=96) == UNSUP
     assert fn(lib, D=32) == UNSUP
     assert fn(lib, Hq=0, Hk=0) == SHAPE
@@ -88,6 +89,10 @@ def test_validation(lib, fn):
     assert fn(lib, gk=G2 + 4) == ALIGN
     assert fn(lib, stride=W + 4) == ALIGN  # 8 bytes of bf16: rows lose 16-byte alignment
     assert fn(lib, dtype=FP32, stride=W + 2) == ALIGN
+    assert fn(lib, dtype=FP16, stride=W + 4) == ALIGN
+    assert fn(lib, dtype=FP8, stride=W + 8) == ALIGN  # 8 bytes of e4m3 per row
+    for dt in (FP16, FP8):  # accepted dtypes reach the pointer checks
+        assert fn(lib, dtype=dt, qkv=P + 8) == ALIGN
     assert lib.qknorm_last_cuda_error() == 0
 
 

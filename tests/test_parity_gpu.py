@@ -102,7 +102,8 @@ def sampled_parity(d, kind, nshards_list=(1,), n_random=256, seed=0):
         run(kind, buf, c, d["gamma_q"], d["gamma_k"], n)
         torch.cuda.synchronize()
         gu.check(gu.stored_bits(buf[idx]), want, x_s, c.dtype, qk, "%s n=%d" % (kind, n))
-        bits = buf.view(torch.int16) if buf.dtype == torch.bfloat16 else buf.view(torch.int32)
+        bits = buf.view(torch.uint8) if buf.dtype == torch.float8_e4m3fn else (
+            buf.view(torch.int16) if buf.element_size() == 2 else buf.view(torch.int32))
         if first is None:
             first = bits
         else:
@@ -188,6 +189,36 @@ def test_layerwise_wide_tokens(dtype, D, Hq, Hk, ns):
             for n in ns]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
+
+
+@pytest.mark.parametrize("dtype", (synth.FP16, synth.FP8))
+@pytest.mark.parametrize("D", synth.STRESS_D)
+def test_low_precision_per_head(dtype, D):
+    c = synth.make_case(333, 32, 8, D, dtype=dtype, seed=50 + D, scale="stress",
+                        zero_frac=0.02, outlier_frac=0.02)
+    full_parity(c, "per_head", what="%s per-head gqa D=%d" % (dtype, D))
+    c = synth.make_case(257, 48, 0, D, dtype=dtype, seed=51 + D)
+    full_parity(c, "per_head", what="%s per-head sweep D=%d" % (dtype, D))
+
+
+@pytest.mark.parametrize("dtype", (synth.FP16, synth.FP8))
+@pytest.mark.parametrize("D", synth.STRESS_D)
+@pytest.mark.parametrize("Hq,Hk", [(32, 8), (64, 8)])
+def test_low_precision_layerwise(dtype, D, Hq, Hk):
+    c = synth.make_case(211, Hq, Hk, D, dtype=dtype, seed=60 + D + Hq, layerwise=True,
+                        scale="lognormal")
+    outs = [full_parity(c, "layerwise", n, what="%s layerwise D=%d n=%d" % (dtype, D, n))[0]
+            for n in (1, 8)]
+    assert np.array_equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("dtype", (synth.FP16, synth.FP8))
+def test_low_precision_full_size_sampled(dtype):
+    d = synth.make_case_torch(16384, device="cuda", seed=70, **dict(synth.GQA, dtype=dtype))
+    sampled_parity(d, "per_head")
+    del d
+    d = synth.make_case_torch(8192, device="cuda", seed=71, **dict(synth.LAYERWISE, dtype=dtype))
+    sampled_parity(d, "layerwise", (1, 8))
 
 
 def test_zero_eps_on_nonzero_rows():
