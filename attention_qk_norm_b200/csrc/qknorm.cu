@@ -9,13 +9,13 @@
 //
 // Per-head (sglang PR #13189, Motivation / Modifications; RMSNorm definition
 // from the SwiftQK review, core_discovery): one sub-warp of LPR lanes owns a
-// (token, head) row of D elements.  Each lane holds D*sizeof/16/LPR 16-byte
-// vectors of the row, sums squares in fp32, and the sub-warp reduces with
+// (token, head) row of D elements.  Each lane holds D/kVec/LPR vectors of
+// the row, sums squares in fp32, and the sub-warp reduces with
 // xor shuffles.  Every thread keeps two rows in flight per iteration and its
 // slice of gamma_q / gamma_k in registers for the whole launch.
 //
 // Layerwise (SwiftQK abstract; review key_machinery): a persistent block
-// walks tokens with a grid stride.  Each thread copies its 16-byte vectors of
+// walks tokens with a grid stride.  Each thread copies its vectors of
 // the next token into a two-stage shared-memory ring with cp.async while it
 // works on the current one.  The per-head partial sums of squares meet in
 // shared memory behind one barrier; then each warp, for the vectors (q, k)
@@ -50,9 +50,13 @@ constexpr int kMaxDevices = 64;
 template <typename TS>
 struct Storage;
 
+// Each storage type moves through memory in 16-byte vectors (type Vec) of
+// kVec elements: 8 for bf16 / fp16, 4 for fp32, 16 for FP8.  (8-byte vectors
+// for FP8, 8 elements like bf16, measured slower on B200.)
 template <>
 struct Storage<__nv_bfloat16> {
-    static constexpr int kVec = 8;  // elements per 16-byte vector
+    using Vec = uint4;
+    static constexpr int kVec = 8;  // elements per vector
     __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
     {
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -76,6 +80,7 @@ struct Storage<__nv_bfloat16> {
 
 template <>
 struct Storage<float> {
+    using Vec = uint4;
     static constexpr int kVec = 4;
     __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[4])
     {
@@ -93,6 +98,7 @@ struct Storage<float> {
 
 template <>
 struct Storage<__half> {
+    using Vec = uint4;
     static constexpr int kVec = 8;
     __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
     {
@@ -116,11 +122,12 @@ struct Storage<__half> {
     }
 };
 
-// FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per vector.
-// Decoded exactly through fp16; encoded round-to-nearest-even, saturating to
-// +-448.  The lower byte of each pair is the earlier element.
+// FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per 16-byte
+// vector.  Decoded exactly through fp16; encoded round-to-nearest-even,
+// saturating to +-448.  The lower byte of each pair is the earlier element.
 template <>
 struct Storage<__nv_fp8_e4m3> {
+    using Vec = uint4;
     static constexpr int kVec = 16;
     __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[16])
     {
@@ -152,9 +159,14 @@ struct Storage<__nv_fp8_e4m3> {
     }
 };
 
-// Streaming (evict-first) 16-byte accesses: each element is touched once.
+// Streaming (evict-first) vector accesses: each element is touched once.
 __device__ __forceinline__ uint4 load_stream(const uint4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void store_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
+
+template <typename V>
+__device__ __forceinline__ V zero_vec();
+template <>
+__device__ __forceinline__ uint4 zero_vec<uint4>() { return make_uint4(0u, 0u, 0u, 0u); }
 
 template <int N>
 __device__ __forceinline__ void load_gamma(const float *__restrict__ g, float (&out)[N])
@@ -189,11 +201,13 @@ __device__ __forceinline__ void pdl_wait_then_release()
     asm volatile("griddepcontrol.launch_dependents;");
 }
 
-// cp.async (16 bytes, L2 only) into shared memory, in commit groups.  Each
-// thread waits only for its own groups (cp.async.wait_group), which the
-// hardware completes; there is no spin loop.
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+// cp.async of one 16-byte vector into shared memory through L2 only (.cg),
+// in commit groups.  Each thread waits only for its own groups
+// (cp.async.wait_group), which the hardware completes; there is no spin loop.
+template <int kBytes>
+__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
 {
+    static_assert(kBytes == 16, "vectors are 16 bytes");
     const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
@@ -232,8 +246,9 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
                     const float *__restrict__ gamma_k, float eps)
 {
     using S = Storage<TS>;
+    using V = typename S::Vec;
     constexpr int kVec = S::kVec;
-    constexpr int kNV = D / kVec;                  // 16-byte vectors per row
+    constexpr int kNV = D / kVec;                  // vectors per row
     constexpr int kLPR = kNV < 32 ? kNV : 32;      // lanes per row
     constexpr int kVPL = kNV / kLPR;               // vectors per lane per row
     constexpr int kEPL = kVPL * kVec;              // elements per lane per row
@@ -277,14 +292,14 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
     // The trip count is the same for every thread, so whole warps reach each
     // shuffle together; rows past the end contribute zeros and store nothing.
     for (uint64_t base = 0; base < rows; base += step) {
-        uint4 x[U][kVPL];
-        uint4 *ptr[U];
+        V x[U][kVPL];
+        V *ptr[U];
 #pragma unroll
         for (int k = 0; k < U; ++k) {
-            ptr[k] = reinterpret_cast<uint4 *>(qkv + t[k] * row_stride + (int64_t)h[k] * D) + lane;
+            ptr[k] = reinterpret_cast<V *>(qkv + t[k] * row_stride + (int64_t)h[k] * D) + lane;
 #pragma unroll
             for (int v = 0; v < kVPL; ++v)
-                x[k][v] = t[k] < T ? load_stream(ptr[k] + v * kLPR) : make_uint4(0u, 0u, 0u, 0u);
+                x[k][v] = t[k] < T ? load_stream(ptr[k] + v * kLPR) : zero_vec<V>();
         }
 #pragma unroll
         for (int k = 0; k < U; ++k) {
@@ -371,8 +386,10 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
                      const float *__restrict__ gamma_k, float eps, float len_q, float len_k)
 {
     using S = Storage<TS>;
+    using V = typename S::Vec;
+    constexpr int kVB = (int)sizeof(V);  // bytes per vector
     constexpr int kVec = S::kVec;
-    constexpr int kNV = D / kVec;     // 16-byte vectors per head
+    constexpr int kNV = D / kVec;     // vectors per head
     constexpr int kLPH = kNV / VPT;   // threads per head
     constexpr int kEPT = VPT * kVec;  // elements per thread
     constexpr int NST = kLayerwiseStages;
@@ -422,10 +439,11 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     // Each thread copies, and later reads, only its own vectors of a stage.
     auto fetch = [&](int64_t tok, int st) {
         if (active && tok < T) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(qkv + tok * row_stride + col0);
+            const V *src = reinterpret_cast<const V *>(qkv + tok * row_stride + col0);
             unsigned char *dst = smem + (size_t)st * span + scol0;
 #pragma unroll
-            for (int v = 0; v < VPT; ++v) cp_async16(dst + (l + v * kLPH) * 16, src + l + v * kLPH);
+            for (int v = 0; v < VPT; ++v)
+                cp_async<kVB>(dst + (l + v * kLPH) * kVB, src + l + v * kLPH);
         }
         cp_async_commit();
     };
@@ -441,12 +459,12 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         // Refill the stage this thread finished with on the previous token.
         fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
         cp_async_wait<NST - 1>();
-        const uint4 *sp = reinterpret_cast<const uint4 *>(smem + (size_t)st * span + scol0);
+        const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
         float s = 0.f;
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
             float f[kVec];
-            S::unpack(active ? sp[l + v * kLPH] : make_uint4(0u, 0u, 0u, 0u), f);
+            S::unpack(active ? sp[l + v * kLPH] : zero_vec<V>(), f);
 #pragma unroll
             for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
         }
@@ -468,7 +486,7 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         const float rk = need_k ? warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane) : 0.f;
         if (active) {
             const float rinv = h < Hq ? rq : rk;
-            uint4 *p = reinterpret_cast<uint4 *>(qkv + t * row_stride + col0);
+            V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
 #pragma unroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec], o[kVec], gv[kVec];
@@ -659,8 +677,8 @@ int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, co
     return launch_per_head_k<TS, D, false>(qkv, T, Hq, Hk, row_stride, g, nullptr, eps, stream);
 }
 
-// A layerwise kernel variant exists when a head splits into whole 16-byte
-// vectors per thread on at most 32 lanes.  Gamma stays in registers up to 32
+// A layerwise kernel variant exists when a head splits into whole vectors
+// per thread on at most 32 lanes.  Gamma stays in registers up to 32
 // elements per thread, else it is read through L1 when scaling.
 template <typename TS, int D, int VPT>
 constexpr bool layerwise_vpt_ok()

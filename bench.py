@@ -555,6 +555,8 @@ PROFILE_CASES = {
                 scale="lognormal", seed=1002),
     "layerwise": dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
                       nshards=8, seed=1003),
+    "per_head_fp8": dict(kind="per_head", T=32768, Hq=32, Hk=8, D=128, dtype="fp8_e4m3",
+                         eps=1e-6, nshards=1, scale="lognormal", seed=1002),
     "layerwise_wide": dict(kind="layerwise", T=8192, Hq=64, Hk=8, D=128, dtype="bf16", eps=1e-6,
                            nshards=8, scale="stress", zero_frac=0.01, outlier_frac=0.01,
                            seed=1004),
