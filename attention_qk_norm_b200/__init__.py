@@ -14,7 +14,12 @@ from ._binding import (  # noqa: F401
     QKNormError,
     load_library,
     qknorm_layerwise,
+    qknorm_layerwise_apply,
+    qknorm_layerwise_partials,
+    qknorm_layerwise_tp,
     qknorm_per_head,
+    tp_allreduce_,
+    tp_full_lengths,
     status_string,
 )
 from .buildlib import LIB_PATH, build  # noqa: F401

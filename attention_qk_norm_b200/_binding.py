@@ -49,6 +49,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.qknorm_per_head.restype = i32
         lib.qknorm_layerwise.argtypes = [vp, i32, i64, i32, i32, i32, i64, vp, vp, f32, i32, vp]
         lib.qknorm_layerwise.restype = i32
+        lib.qknorm_layerwise_partials.argtypes = [vp, i32, i64, i32, i32, i32, i64, vp, vp]
+        lib.qknorm_layerwise_partials.restype = i32
+        lib.qknorm_layerwise_apply.argtypes = [vp, i32, i64, i32, i32, i32, i64, vp, vp, vp,
+                                               i64, i64, f32, vp]
+        lib.qknorm_layerwise_apply.restype = i32
         lib.qknorm_status_string.argtypes = [i32]
         lib.qknorm_status_string.restype = ctypes.c_char_p
         lib.qknorm_last_cuda_error.argtypes = []
@@ -107,12 +112,12 @@ def _gamma_ptr(g, name):
     return ctypes.c_void_p(g.data_ptr())
 
 
-def _device_check(qkv, *gammas):
+def _device_check(qkv, *others):
     if not qkv.is_cuda:
         raise ValueError("qkv must be a CUDA tensor (QK-Norm runs only on the GPU)")
-    for g in gammas:
+    for g in others:
         if g is not None and g.device != qkv.device:
-            raise ValueError("gamma must live on the same device as qkv")
+            raise ValueError("gamma and sums must live on the same device as qkv")
 
 
 def qknorm_per_head(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, row_stride=None, stream=None):
@@ -138,3 +143,75 @@ def qknorm_layerwise(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, nshards=1, row_strid
         int(nshards), _stream_ptr(qkv, stream))
     _check("qknorm_layerwise", rc)
     return qkv
+
+
+def qknorm_layerwise_partials(qkv, Hq, Hk, D, partials=None, row_stride=None, stream=None):
+    """This rank's per-token fp32 sums of squares, ``[T, 2]`` (q, k) float32.
+
+    ``qkv`` holds this rank's heads (Hq query, Hk key/value) in the fused
+    layout; it is only read.  ``partials`` may be passed to reuse memory."""
+    import torch
+
+    _device_check(qkv)
+    T, stride = _rows(qkv, row_stride)
+    if partials is None:
+        partials = torch.empty((T, 2), dtype=torch.float32, device=qkv.device)
+    if partials.dtype != torch.float32 or not partials.is_contiguous() or partials.numel() < 2 * T:
+        raise ValueError("partials must be a contiguous float32 tensor of 2*T elements")
+    rc = load_library().qknorm_layerwise_partials(
+        ctypes.c_void_p(qkv.data_ptr()), _dtype_code(qkv), T, Hq, Hk, D, stride,
+        ctypes.c_void_p(partials.data_ptr()), _stream_ptr(qkv, stream))
+    _check("qknorm_layerwise_partials", rc)
+    return partials
+
+
+def qknorm_layerwise_apply(qkv, Hq, Hk, D, gamma_q, gamma_k, sums, len_q, len_k, eps,
+                           row_stride=None, stream=None):
+    """Scale this rank's q / k columns in place by the inverse RMS that the
+    summed partials ``sums`` ([T, 2] float32) and the full lengths give."""
+    import torch
+
+    _device_check(qkv, gamma_q, gamma_k, sums)
+    T, stride = _rows(qkv, row_stride)
+    if sums.dtype != torch.float32 or not sums.is_contiguous() or sums.numel() < 2 * T:
+        raise ValueError("sums must be a contiguous float32 tensor of 2*T elements")
+    rc = load_library().qknorm_layerwise_apply(
+        ctypes.c_void_p(qkv.data_ptr()), _dtype_code(qkv), T, Hq, Hk, D, stride,
+        _gamma_ptr(gamma_q, "gamma_q"), _gamma_ptr(gamma_k, "gamma_k"),
+        ctypes.c_void_p(sums.data_ptr()), int(len_q), int(len_k), float(eps),
+        _stream_ptr(qkv, stream))
+    _check("qknorm_layerwise_apply", rc)
+    return qkv
+
+
+def tp_allreduce_(partials, group=None) -> int:
+    """Sum ``partials`` over the ranks of ``group`` in place (one all-reduce;
+    nothing without an initialised process group); returns the group size."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return 1
+    world = dist.get_world_size(group)
+    if world > 1:
+        dist.all_reduce(partials, op=dist.ReduceOp.SUM, group=group)
+    return world
+
+
+def tp_full_lengths(Hq, Hk, D, world):
+    """Full q / k vector lengths when every rank holds Hq and Hk heads."""
+    return Hq * D * world, Hk * D * world
+
+
+def qknorm_layerwise_tp(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, group=None, row_stride=None):
+    """Layerwise QK-Norm across a tensor-parallel group, in place.
+
+    Every rank of ``group`` (torch.distributed; a single process when it is
+    not initialised) holds ``Hq`` query and ``Hk`` key/value heads of every
+    token.  Steps: this rank's partial sums (qknorm_layerwise_partials), one
+    all-reduce of the 2*T scalars over the group, and the scaling
+    (qknorm_layerwise_apply) with the full vector lengths."""
+    partials = qknorm_layerwise_partials(qkv, Hq, Hk, D, row_stride=row_stride)
+    world = tp_allreduce_(partials, group)
+    len_q, len_k = tp_full_lengths(Hq, Hk, D, world)
+    return qknorm_layerwise_apply(qkv, Hq, Hk, D, gamma_q, gamma_k, partials, len_q, len_k, eps,
+                                  row_stride=row_stride)

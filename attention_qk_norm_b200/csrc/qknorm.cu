@@ -340,8 +340,8 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
 // --------------------------------------------------------------- layerwise --
 constexpr int kLayerwiseStages = 2;
 
-// Inverse RMS of one vector of `nh` heads from their partials part[0..nh),
-// computed by one whole warp; every lane returns the same value.
+// Sum of squares of one vector of `nh` heads from their partials
+// part[0..nh), computed by one whole warp; every lane returns the same value.
 //
 // The reduction tree is fixed by nh alone.  Let p be the largest power of two
 // dividing nh and u = min(p, 32) the lanes used: lane i sums heads
@@ -351,8 +351,7 @@ constexpr int kLayerwiseStages = 2;
 // below distance u/n form each shard's partial S_r from that shard's heads
 // only, and the remaining ones are the scalar combine of S_0..S_{n-1}.  So
 // the result does not depend on n, bit for bit.
-__device__ __forceinline__ float warp_rinv(const float *part, int nh, int nshards, float len,
-                                           float eps, int lane)
+__device__ __forceinline__ float warp_sumsq(const float *part, int nh, int nshards, int lane)
 {
     if (nh == 0) return 0.f;
     const int p2 = nh & (-nh);
@@ -366,9 +365,17 @@ __device__ __forceinline__ float warp_rinv(const float *part, int nh, int nshard
         v += __shfl_xor_sync(0xffffffffu, v, o);
     for (int o = per_shard; o < used; o <<= 1)  // combine of the shard scalars
         v += __shfl_xor_sync(0xffffffffu, v, o);
-    v = __shfl_sync(0xffffffffu, v, 0);
-    return rsqrtf(v / len + eps);
+    return __shfl_sync(0xffffffffu, v, 0);
 }
+
+// What a layerwise launch does with a token.
+//   kFused:    partial sums, scalar combine, inverse RMS and scaling, in place.
+//   kPartials: only this rank's two fp32 sums of squares (its q heads, its k
+//              heads), written to aux[2t], aux[2t+1]; the data is not written.
+//   kApply:    only the scaling, by 1/sqrt(aux[2t]/len_q + eps) for q and
+//              1/sqrt(aux[2t+1]/len_k + eps) for k, where aux holds the sums
+//              over all ranks and len_q, len_k the full vector lengths.
+enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 
 // A token's heads are split over the CL blocks of a thread-block cluster
 // (CL = 1 for a plain launch): block c of a cluster owns heads
@@ -379,11 +386,12 @@ __device__ __forceinline__ float warp_rinv(const float *part, int nh, int nshard
 // `heads` fp32 head partials (alternating per token).  With CL > 1 every block
 // writes its head partials into all blocks of its cluster (distributed shared
 // memory) before the cluster barrier, so each block then holds all of them.
-template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster>
+template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode>
 __global__ void __launch_bounds__(1024)
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                      int nshards, const float *__restrict__ gamma_q,
-                     const float *__restrict__ gamma_k, float eps, float len_q, float len_k)
+                     const float *__restrict__ gamma_k, float eps, float len_q, float len_k,
+                     float *__restrict__ aux)
 {
     using S = Storage<TS>;
     using V = typename S::Vec;
@@ -425,7 +433,7 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     float g[kGammaRegs ? kEPT : 1];
 #pragma unroll
     for (int e = 0; e < (kGammaRegs ? kEPT : 1); ++e) g[e] = 0.f;
-    if (kGammaRegs && active) {
+    if (kGammaRegs && kMode != kPartials && active) {
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
             float t4[kVec];
@@ -453,38 +461,57 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     // cluster is running: meet once before the first remote write.  (The last
     // remote write of the loop precedes its final cluster barrier, so no block
     // exits while another may still write into it.)
-    if constexpr (kCluster) cooperative_groups::this_cluster().sync();
+    if constexpr (kCluster && kMode != kApply) cooperative_groups::this_cluster().sync();
     int st = 0, pb = 0;
     for (int64_t t = first; t < T; t += stride) {
         // Refill the stage this thread finished with on the previous token.
         fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
         cp_async_wait<NST - 1>();
         const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
-        float s = 0.f;
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) {
-            float f[kVec];
-            S::unpack(active ? sp[l + v * kLPH] : zero_vec<V>(), f);
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
-        }
-        s = group_sum<kLPH>(s);
-        // Partials alternate between two buffers: a warp still reading this
-        // token's buffer cannot meet a write of the next token's, which only
-        // starts after the next barrier (of the block, or of the cluster).
-        float *pp = part + pb * heads;
-        if constexpr (kCluster) {
-            cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
-            if (active && l == 0)
-                for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(pp + h, r) = s;
-            cluster.sync();
+        float rq = 0.f, rk = 0.f;
+        if constexpr (kMode == kApply) {
+            // Sums over all ranks come in; no exchange inside the launch.
+            if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) / len_q + eps);
+            if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) / len_k + eps);
         } else {
-            if (active && l == 0) pp[h] = s;
-            __syncthreads();
+            float s = 0.f;
+    #pragma unroll
+            for (int v = 0; v < VPT; ++v) {
+                float f[kVec];
+                S::unpack(active ? sp[l + v * kLPH] : zero_vec<V>(), f);
+    #pragma unroll
+                for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
+            }
+            s = group_sum<kLPH>(s);
+            // Partials alternate between two buffers: a warp still reading this
+            // token's buffer cannot meet a write of the next token's, which only
+            // starts after the next barrier (of the block, or of the cluster).
+            float *pp = part + pb * heads;
+            if constexpr (kCluster) {
+                cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+                if (active && l == 0)
+                    for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(pp + h, r) = s;
+                cluster.sync();
+            } else {
+                if (active && l == 0) pp[h] = s;
+                __syncthreads();
+            }
+            if constexpr (kMode == kPartials) {
+                // One warp of the cluster's first block writes this rank's sums.
+                if (threadIdx.x < 32 && crank == 0) {
+                    const float sq = warp_sumsq(pp, Hq, 1, lane);
+                    const float sk = warp_sumsq(pp + Hq, Hk, 1, lane);
+                    if (lane == 0) {
+                        aux[2 * t] = sq;
+                        aux[2 * t + 1] = sk;
+                    }
+                }
+            } else {
+                if (need_q) rq = rsqrtf(warp_sumsq(pp, Hq, nshards, lane) / len_q + eps);
+                if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, Hk, nshards, lane) / len_k + eps);
+            }
         }
-        const float rq = need_q ? warp_rinv(pp, Hq, nshards, len_q, eps, lane) : 0.f;
-        const float rk = need_k ? warp_rinv(pp + Hq, Hk, nshards, len_k, eps, lane) : 0.f;
-        if (active) {
+        if (kMode != kPartials && active) {
             const float rinv = h < Hq ? rq : rk;
             V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
 #pragma unroll
@@ -693,12 +720,13 @@ constexpr bool layerwise_gamma_regs()
     return VPT * Storage<TS>::kVec <= 32;
 }
 
-template <typename TS, int D, int VPT, bool kCluster>
+template <typename TS, int D, int VPT, bool kCluster, int kMode>
 int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
                          const float *gq, const float *gk, float eps, int nshards, int threads,
-                         int cluster, cudaStream_t stream)
+                         int cluster, float len_q, float len_k, float *aux, cudaStream_t stream)
 {
-    auto kern = qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>(), kCluster>;
+    auto kern =
+        qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>(), kCluster, kMode>;
     static KernelCache kc;
     const int heads = Hq + Hk;
     const size_t span = (size_t)(heads / cluster) * D * sizeof(TS);
@@ -737,11 +765,9 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
     }
     if (cap < 1) return QKN_ERR_UNSUPPORTED;
     const int64_t clusters = T < cap ? T : cap;
-    const float len_q = (float)((int64_t)Hq * D);  // exact: spans are < 2^24 elements
-    const float len_k = (float)((int64_t)Hk * D);
     return launch_pdl(kern, (unsigned)(clusters * cluster), threads, smem, stream,
                       (unsigned)cluster, static_cast<TS *>(qkv), row_stride, T, Hq, Hk, nshards,
-                      gq, gk, eps, len_q, len_k);
+                      gq, gk, eps, len_q, len_k, aux);
 }
 
 // Launch shape.  First choice: the smallest cluster (1, 2, 4 or 8 blocks,
@@ -752,10 +778,15 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 constexpr int kLayerwiseTargetThreads = 256;
 constexpr int kMaxCluster = 8;
 
-template <typename TS, int D>
+// len_q, len_k: the normalised lengths (the full vectors; for kFused and
+// kPartials they are this launch's own Hq*D and Hk*D).
+template <typename TS, int D, int kMode = kFused>
 int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
-                     const float *gk, float eps, int nshards, cudaStream_t stream)
+                     const float *gk, float eps, int nshards, cudaStream_t stream,
+                     float len_q = -1.f, float len_k = -1.f, float *aux = nullptr)
 {
+    if (len_q < 0.f) len_q = (float)((int64_t)Hq * D);  // exact: spans are < 2^24 elements
+    if (len_k < 0.f) len_k = (float)((int64_t)Hk * D);
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kVec = Storage<TS>::kVec;
     const int64_t heads = Hq + Hk;
@@ -788,12 +819,13 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
         if constexpr (layerwise_vpt_ok<TS, D, V>()) {                                          \
             if constexpr (layerwise_gamma_regs<TS, V>()) {                                     \
                 if (cluster > 1)                                                               \
-                    return launch_layerwise_vpt<TS, D, V, true>(qkv, T, Hq, Hk, row_stride,    \
-                                                                gq, gk, eps, nshards, threads, \
-                                                                cluster, stream);              \
+                    return launch_layerwise_vpt<TS, D, V, true, kMode>(                        \
+                        qkv, T, Hq, Hk, row_stride, gq, gk, eps, nshards, threads, cluster,    \
+                        len_q, len_k, aux, stream);                                            \
             }                                                                                  \
-            return launch_layerwise_vpt<TS, D, V, false>(qkv, T, Hq, Hk, row_stride, gq, gk,   \
-                                                         eps, nshards, threads, 1, stream);    \
+            return launch_layerwise_vpt<TS, D, V, false, kMode>(                               \
+                qkv, T, Hq, Hk, row_stride, gq, gk, eps, nshards, threads, 1, len_q, len_k,    \
+                aux, stream);                                                                  \
         }                                                                                      \
         break;
     switch (chosen) {
@@ -836,7 +868,15 @@ struct PerHead {
 };
 struct Layerwise {
     template <typename TS, int D, typename... A>
-    static int run(A... a) { return launch_layerwise<TS, D>(a...); }
+    static int run(A... a) { return launch_layerwise<TS, D, kFused>(a...); }
+};
+struct LayerwisePartials {
+    template <typename TS, int D, typename... A>
+    static int run(A... a) { return launch_layerwise<TS, D, kPartials>(a...); }
+};
+struct LayerwiseApply {
+    template <typename TS, int D, typename... A>
+    static int run(A... a) { return launch_layerwise<TS, D, kApply>(a...); }
 };
 
 }  // namespace
@@ -867,6 +907,41 @@ int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int
                                nshards, static_cast<cudaStream_t>(stream));
 }
 
+int qknorm_layerwise_partials(const void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                              int64_t row_stride, float *partials, void *stream)
+{
+    bool done = false;
+    // The weights play no part here; validate the buffer as if they were set.
+    const float *no_gamma = reinterpret_cast<const float *>(qkv);
+    int rc = validate(qkv, dtype, T, Hq, Hk, D, row_stride, Hq > 0 ? no_gamma : nullptr,
+                      Hk > 0 ? no_gamma : nullptr, 0.f, &done);
+    if (rc != QKN_OK || done) return rc;
+    if (partials == nullptr) return QKN_ERR_NULL;
+    if (((uintptr_t)partials & 7u) != 0) return QKN_ERR_ALIGN;
+    return dispatch<LayerwisePartials>(dtype, D, const_cast<void *>(qkv), T, Hq, Hk, row_stride,
+                                       (const float *)nullptr, (const float *)nullptr, 0.f, 1,
+                                       static_cast<cudaStream_t>(stream), -1.f, -1.f, partials);
+}
+
+int qknorm_layerwise_apply(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                           int64_t row_stride, const float *gamma_q, const float *gamma_k,
+                           const float *sums, int64_t len_q, int64_t len_k, float eps,
+                           void *stream)
+{
+    bool done = false;
+    const int rc = validate(qkv, dtype, T, Hq, Hk, D, row_stride, gamma_q, gamma_k, eps, &done);
+    if (rc != QKN_OK) return rc;
+    if ((Hq > 0 && len_q < (int64_t)Hq * D) || (Hk > 0 && len_k < (int64_t)Hk * D) ||
+        len_q > (1 << 24) || len_k > (1 << 24))
+        return QKN_ERR_SHAPE;
+    if (done) return QKN_OK;
+    if (sums == nullptr) return QKN_ERR_NULL;
+    if (((uintptr_t)sums & 7u) != 0) return QKN_ERR_ALIGN;
+    return dispatch<LayerwiseApply>(dtype, D, qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps,
+                                    1, static_cast<cudaStream_t>(stream), (float)len_q,
+                                    (float)len_k, const_cast<float *>(sums));
+}
+
 const char *qknorm_status_string(int status)
 {
     switch (status) {
@@ -884,6 +959,6 @@ const char *qknorm_status_string(int status)
 
 int qknorm_last_cuda_error(void) { return g_last_cuda_error; }
 
-int qknorm_version(void) { return 101; }
+int qknorm_version(void) { return 102; }
 
 }  // extern "C"

@@ -116,13 +116,48 @@ int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int
                      const float *gamma_q, const float *gamma_k, float eps, int nshards,
                      void *stream);
 
+/*
+ * Tensor-parallel layerwise QK-Norm, the two rank-local steps.  Sources: the
+ * SwiftQK review (key_machinery and core_discovery: each rank reduces its
+ * shard to a local sum of squares, the ranks exchange only these scalars, and
+ * every element is scaled by the global factor 1/sqrt(S_global/H + eps)) and
+ * the "combined QKV projection" lesson (tensor-parallel follow-up: each rank
+ * holds its share of the Q heads and of the K/V heads).  A rank's buffer is
+ * the fused QKV of its own heads: Hq query heads and Hk key/value heads here
+ * are this rank's counts, in the layout described at the top.
+ *
+ * qknorm_layerwise_partials writes, for every token t, the fp32 sum of
+ * squares of this rank's q columns to partials[2t] and of its k columns to
+ * partials[2t+1] (0 when the rank has no such heads).  partials is
+ * caller-owned device memory of 2*T floats, 8-byte aligned; qkv is only read.
+ * The sums use the same fixed reduction tree as qknorm_layerwise.
+ *
+ * The caller then sums the partials over the ranks (for instance one
+ * all-reduce of 2*T floats) and calls qknorm_layerwise_apply with the sums:
+ * it scales this rank's q columns by gamma_q[j] / sqrt(sums[2t]/len_q + eps)
+ * and its k columns by gamma_k[j] / sqrt(sums[2t+1]/len_k + eps), in place,
+ * where len_q and len_k are the FULL q and k vector lengths over all ranks
+ * (at least Hq*D and Hk*D, at most 2^24, else QKN_ERR_SHAPE) and gamma_q /
+ * gamma_k this rank's slices (Hq*D and Hk*D floats).  sums is 2*T floats,
+ * 8-byte aligned.  With a single rank, the two calls give exactly the output
+ * of qknorm_layerwise.  Arguments and errors are otherwise those above.
+ */
+int qknorm_layerwise_partials(const void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                              int64_t row_stride, float *partials, void *stream);
+
+int qknorm_layerwise_apply(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                           int64_t row_stride, const float *gamma_q, const float *gamma_k,
+                           const float *sums, int64_t len_q, int64_t len_k, float eps,
+                           void *stream);
+
 /* Static English text for a qkn_status value (never NULL). */
 const char *qknorm_status_string(int status);
 
 /* cudaError_t of the calling thread's last QKN_ERR_CUDA (0 if none). */
 int qknorm_last_cuda_error(void);
 
-/* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3). */
+/* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3, 1.02 the
+ * tensor-parallel layerwise steps). */
 int qknorm_version(void);
 
 #ifdef __cplusplus

@@ -37,7 +37,8 @@ def declared_symbols():
 def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
     assert set(names) == {"qknorm_per_head", "qknorm_layerwise", "qknorm_status_string",
-                          "qknorm_last_cuda_error", "qknorm_version"}
+                          "qknorm_last_cuda_error", "qknorm_version", "qknorm_layerwise_partials",
+                          "qknorm_layerwise_apply"}
     for n in names:
         assert hasattr(lib, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", qbuild.LIB_PATH], capture_output=True,
@@ -47,7 +48,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.qknorm_version() == 101
+    assert lib.qknorm_version() == 102
     for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS):
         s = lib.qknorm_status_string(code).decode()
         assert s and s != "unknown status"
@@ -111,6 +112,33 @@ def test_layerwise_nshards(lib):
     assert lw(lib, T=0, n=3) == NSHARDS  # checked even when there is nothing to do
     assert lw(lib, T=0, n=8, qkv=None) == OK
     assert lw(lib, n=8, qkv=P + 8) == ALIGN  # valid nshards, reaches later checks
+
+
+def test_tensor_parallel_steps_validation(lib):
+    W = (32 + 16) * 128
+    part = lib.qknorm_layerwise_partials
+    assert part(P, BF16, 4, 32, 8, 128, W, None, None) == NULL
+    assert part(P, BF16, 4, 32, 8, 128, W, G1 + 4, None) == ALIGN
+    assert part(P + 8, BF16, 4, 32, 8, 128, W, G1, None) == ALIGN
+    assert part(P, BF16, 4, 32, 8, 96, W, G1, None) == UNSUP
+    assert part(None, BF16, 0, 32, 8, 128, W, None, None) == OK  # T == 0: nothing to do
+    app = lib.qknorm_layerwise_apply
+    args = (BF16, 4, 32, 8, 128, W, G1, G2)
+    assert app(P, *args, None, 4 * 4096, 4 * 1024, 1e-6, None) == NULL
+    S = 0x300000  # 8-byte aligned; S + 4 is not
+    assert app(P, *args, S + 4, 4 * 4096, 4 * 1024, 1e-6, None) == ALIGN
+    assert app(P, *args, S, 4095, 1024, 1e-6, None) == SHAPE  # below this rank's Hq*D
+    assert app(P, *args, S, 4096, 1023, 1e-6, None) == SHAPE
+    assert app(P, *args, S, 1 << 25, 1024, 1e-6, None) == SHAPE
+    assert app(P, *args, S, 4096, 1024, -1.0, None) == EPS
+    assert app(P, BF16, 4, 32, 8, 128, W, None, G2, S, 4096, 1024, 1e-6, None) == NULL
+    assert app(None, BF16, 0, 32, 8, 128, W, None, None, None, 4096, 1024, 1e-6, None) == OK
+    assert lib.qknorm_last_cuda_error() == 0
+
+
+def test_tp_lengths():
+    assert qkn.tp_full_lengths(8, 2, 128, 4) == (4096, 1024)
+    assert qkn.tp_allreduce_(None) == 1  # no process group: a single rank
 
 
 def test_binding_rejects_host_tensors():

@@ -35,6 +35,50 @@ def _worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def _tp_worker(rank, world, port, q):
+    """Each rank sums squares over its head shard of the same tokens; one
+    all-reduce must give the full-vector sums, and the full lengths must be
+    the local ones times the group size."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import attention_qk_norm_b200 as qkn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    T, Hq, Hk, D = 5, 8, 4, 16
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((T, (Hq + Hk) * D))
+    xq, xk = x[:, :Hq * D], x[:, Hq * D:]
+    hq, hk = Hq // world, Hk // world
+    mine_q = xq[:, rank * hq * D:(rank + 1) * hq * D]
+    mine_k = xk[:, rank * hk * D:(rank + 1) * hk * D]
+    partials = torch.tensor(np.stack([(mine_q ** 2).sum(1), (mine_k ** 2).sum(1)], 1))
+    got = qkn.tp_allreduce_(partials)
+    full = np.stack([(xq ** 2).sum(1), (xk ** 2).sum(1)], 1)
+    q.put((rank, got, bool(np.allclose(partials.numpy(), full, rtol=1e-12)),
+           qkn.tp_full_lengths(hq, hk, D, got)))
+    dist.destroy_process_group()
+
+
+def test_tensor_parallel_allreduce_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_tp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, ok, lens in out:
+        assert got == world and ok and lens == (8 * 16, 4 * 16)
+
+
 def test_two_gloo_ranks_barrier_and_max():
     world = 2
     ctx = mp.get_context("spawn")

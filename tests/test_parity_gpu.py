@@ -261,3 +261,66 @@ def test_errors_leave_buffer_untouched():
     assert e.value.status == -5
     torch.cuda.synchronize()
     assert torch.equal(full.view(torch.int16), before.view(torch.int16))
+
+
+# ------------------------------------------- tensor-parallel layerwise steps --
+def _rank_columns(c, n, r):
+    """Global columns of rank r's fused buffer when heads are split in n
+    contiguous groups (its Q heads, then its K heads, then its V heads)."""
+    hq, hk, D = c.Hq // n, c.Hk // n, c.D
+    q = np.arange(r * hq * D, (r + 1) * hq * D)
+    k = c.Hq * D + np.arange(r * hk * D, (r + 1) * hk * D)
+    v = (c.Hq + c.Hk) * D + np.arange(r * hk * D, (r + 1) * hk * D)
+    return np.concatenate([q, k, v]), hq, hk
+
+
+@pytest.mark.parametrize("Hq,Hk,D,dtype", [(32, 8, 128, synth.BF16), (64, 8, 256, synth.FP32),
+                                           (32, 8, 64, synth.FP8), (16, 8, 128, synth.FP16)])
+@pytest.mark.parametrize("n", (1, 2, 4, 8))
+def test_tensor_parallel_steps_emulated(Hq, Hk, D, dtype, n):
+    """n ranks emulated one after another on one GPU: each rank's partial sums,
+    their sum (standing in for the all-reduce), each rank's scaling; the
+    reassembled result must match the float64 oracle of the whole vectors."""
+    c = synth.make_case(123, Hq, Hk, D, dtype=dtype, seed=80 + n + D, layerwise=True,
+                        scale="lognormal")
+    W = (Hq + 2 * Hk) * D
+    locals_, sums = [], None
+    for r in range(n):
+        cols, hq, hk = _rank_columns(c, n, r)
+        sub = synth.Case(np.ascontiguousarray(c.qkv[:, cols]),
+                         c.gamma_q[r * hq * D:(r + 1) * hq * D],
+                         c.gamma_k[r * hk * D:(r + 1) * hk * D], c.T, hq, hk, D,
+                         (hq + 2 * hk) * D, dtype, c.eps, True)
+        buf, gq, gk = gu.to_device(sub)
+        part = qkn.qknorm_layerwise_partials(buf, hq, hk, D)
+        sums = part.clone() if sums is None else sums + part
+        locals_.append((cols, sub, buf, gq, gk))
+    out = c.qkv.copy()
+    for cols, sub, buf, gq, gk in locals_:
+        qkn.qknorm_layerwise_apply(buf, sub.Hq, sub.Hk, D, gq, gk, sums, Hq * D, Hk * D, c.eps)
+        torch.cuda.synchronize()
+        out[:, cols] = gu.stored_bits(buf)
+    want = gu.oracle_out(c, "layerwise", c.qkv, c.T)
+    gu.check(out, want, c.qkv, dtype, (Hq + Hk) * D, "tp n=%d" % n)
+    assert out.shape[1] == W
+    if n == 1:  # a single rank is exactly the fused kernel
+        full, gq, gk = gu.to_device(c)
+        qkn.qknorm_layerwise(full, Hq, Hk, D, gq, gk, c.eps)
+        torch.cuda.synchronize()
+        assert np.array_equal(gu.stored_bits(full), out)
+        x, gq, gk = gu.to_device(c)
+        qkn.qknorm_layerwise_tp(x, Hq, Hk, D, gq, gk, c.eps)  # no process group: one rank
+        torch.cuda.synchronize()
+        assert np.array_equal(gu.stored_bits(x), out)
+
+
+def test_tensor_parallel_partials_leave_buffer_untouched():
+    c = synth.make_case(77, 32, 8, 128, seed=90, layerwise=True)
+    buf, _, _ = gu.to_device(c)
+    part = qkn.qknorm_layerwise_partials(buf, 32, 8, 128)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.stored_bits(buf), c.qkv)
+    x = gu.as_f64(c.qkv, c.dtype)
+    want = np.stack([(x[:, :4096] ** 2).sum(1), (x[:, 4096:5120] ** 2).sum(1)], 1)
+    got = part.cpu().numpy().astype(np.float64)
+    assert np.allclose(got, want, rtol=1e-5, atol=0)
