@@ -207,7 +207,7 @@ class Workload:
         self.w = w
         d = synth.make_case_torch(w["T"], w["Hq"], w["Hk"], w["D"], device=device,
                                   dtype=w["dtype"], seed=w["seed"], eps=w["eps"],
-                                  layerwise=w["kind"] == "layerwise",
+                                  layerwise=w["kind"] != "per_head",
                                   scale=w.get("scale"), zero_frac=w.get("zero_frac", 0.0),
                                   outlier_frac=w.get("outlier_frac", 0.0))
         self.gq, self.gk = d["gamma_q"], d["gamma_k"]
@@ -229,6 +229,16 @@ class Workload:
             self.i += 1
         if w["kind"] == "per_head":
             qkn.qknorm_per_head(buf, w["Hq"], w["Hk"], w["D"], self.gq, self.gk, w["eps"])
+        elif w["kind"] == "layerwise_tp":
+            # The two rank-local tensor-parallel steps of one rank (no peers,
+            # so the all-reduce between them is empty).
+            if getattr(self, "partials", None) is None:
+                import torch
+
+                self.partials = torch.empty((w["T"], 2), dtype=torch.float32, device=buf.device)
+            qkn.qknorm_layerwise_partials(buf, w["Hq"], w["Hk"], w["D"], partials=self.partials)
+            qkn.qknorm_layerwise_apply(buf, w["Hq"], w["Hk"], w["D"], self.gq, self.gk,
+                                       self.partials, w["Hq"] * w["D"], w["Hk"] * w["D"], w["eps"])
         else:
             qkn.qknorm_layerwise(buf, w["Hq"], w["Hk"], w["D"], self.gq, self.gk, w["eps"],
                                  nshards=w["nshards"])
@@ -297,6 +307,10 @@ def extra_workloads():
             out.append(("layerwise n=%d" % n, dict(kind="layerwise", T=T, Hq=32, Hk=8, D=128,
                                                     dtype="bf16", eps=1e-6, nshards=n,
                                                     seed=2300 + T)))
+    for T in (4096, 8192):
+        out.append(("layerwise tp steps, 1 rank", dict(kind="layerwise_tp", T=T, Hq=32, Hk=8,
+                                                       D=128, dtype="bf16", eps=1e-6, nshards=1,
+                                                       seed=2700 + T)))
     for dt in (synth.FP16, synth.FP8):
         out.append(("gqa fused 32q/8kv %s" % dt, dict(kind="per_head", T=16384, Hq=32, Hk=8,
                                                       D=128, dtype=dt, eps=1e-6, nshards=1,
