@@ -881,6 +881,41 @@ struct LayerwiseApply {
 
 }  // namespace
 
+
+// ------------------------------------------- entry point without allocation --
+// Library-owned scratch for qknorm_layerwise_noalloc: the per-token partial
+// sums (two fp32 per token) that the two tensor-parallel steps pass between
+// them.  Every GPU that loads the library holds this array until the process
+// exits.  Host code must not use the symbol's address directly: on the host
+// it names a stand-in, not device memory, so the device address is looked up
+// once per device with cudaGetSymbolAddress.
+constexpr int64_t kNoAllocMaxTokens = 65536;  // 512 KiB of partial sums
+static __device__ __align__(256) float g_noalloc_partials[2 * kNoAllocMaxTokens];
+
+namespace {
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_partials on the current device; the first call
+// on a device looks it up (with that device current).
+int noalloc_scratch(float **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return QKN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return QKN_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
@@ -942,6 +977,28 @@ int qknorm_layerwise_apply(void *qkv, int dtype, int64_t T, int Hq, int Hk, int 
                                     (float)len_k, const_cast<float *>(sums));
 }
 
+int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                             int64_t row_stride, const float *gamma_q, const float *gamma_k,
+                             float eps, void *stream)
+{
+    bool done = false;
+    int rc = validate(qkv, dtype, T, Hq, Hk, D, row_stride, gamma_q, gamma_k, eps, &done);
+    if (rc != QKN_OK) return rc;
+    if (T > kNoAllocMaxTokens) return QKN_ERR_TOO_LARGE;
+    if (done) return QKN_OK;
+    float *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != QKN_OK) return rc;
+    // Every entry the second step reads is written by the first step of this
+    // call, so the scratch needs no clearing.
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rc = dispatch<LayerwisePartials>(dtype, D, qkv, T, Hq, Hk, row_stride, (const float *)nullptr,
+                                     (const float *)nullptr, 0.f, 1, s, -1.f, -1.f, scratch);
+    if (rc != QKN_OK) return rc;
+    return dispatch<LayerwiseApply>(dtype, D, qkv, T, Hq, Hk, row_stride, gamma_q, gamma_k, eps,
+                                    1, s, (float)((int64_t)Hq * D), (float)((int64_t)Hk * D),
+                                    scratch);
+}
+
 const char *qknorm_status_string(int status)
 {
     switch (status) {
@@ -953,6 +1010,8 @@ const char *qknorm_status_string(int status)
     case QKN_ERR_UNSUPPORTED: return "unsupported dtype, head_dim, or token span too wide for one block";
     case QKN_ERR_CUDA: return "CUDA runtime error (see qknorm_last_cuda_error)";
     case QKN_ERR_EPS: return "eps must be finite and >= 0";
+    case QKN_ERR_TOO_LARGE:
+        return "T exceeds the 65536 tokens of qknorm_layerwise_noalloc's static scratch";
     default: return "unknown status";
     }
 }

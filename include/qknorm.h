@@ -73,7 +73,8 @@ typedef enum {
     QKN_ERR_NSHARDS = -4,     /* nshards not in {1,2,4,8} or not dividing heads */
     QKN_ERR_UNSUPPORTED = -5, /* dtype or head_dim not built, token too wide    */
     QKN_ERR_CUDA = -6,        /* CUDA runtime error on this call                */
-    QKN_ERR_EPS = -7          /* eps negative or not finite                     */
+    QKN_ERR_EPS = -7,         /* eps negative or not finite                     */
+    QKN_ERR_TOO_LARGE = -8    /* T beyond qknorm_layerwise_noalloc's scratch    */
 } qkn_status;
 
 /*
@@ -149,6 +150,35 @@ int qknorm_layerwise_apply(void *qkv, int dtype, int64_t T, int Hq, int Hk, int 
                            int64_t row_stride, const float *gamma_q, const float *gamma_k,
                            const float *sums, int64_t len_q, int64_t len_k, float eps,
                            void *stream);
+
+/*
+ * Layerwise QK-Norm that allocates nothing (no counterpart in the paper: it
+ * exists for callers, not for the method).  Some callers cannot allocate GPU
+ * memory when they call in: a runtime that hands out memory only from its
+ * own fixed pool, an embedding application that forbids allocations on its
+ * hot path, or code that runs while an allocator lock is held.  This entry
+ * point gives them the result of qknorm_layerwise(..., nshards = 1, ...) -- same
+ * arguments except nshards -- computed with the two tensor-parallel steps
+ * above for a single rank, whose partial sums live in a static device array
+ * inside the library instead of caller memory.  The caller still passes and
+ * owns qkv and the weights.
+ *
+ * Limits and sharing:
+ * - T may be at most 65536 (the array holds 2 * 65536 floats, 512 KiB, which
+ *   every GPU that loads the library keeps until the process exits); larger T
+ *   returns QKN_ERR_TOO_LARGE and launches nothing.
+ * - The first call on a device looks up the array's device address (with that
+ *   device current) and caches it; make that first call before any stream
+ *   capture on the device.
+ * - All calls share the one array per device.  Calls whose work overlaps on
+ *   the GPU (other streams, or other host threads' streams) race on it and
+ *   give wrong results; calls ordered on one stream are fine.  Every partial
+ *   sum a call reads is written earlier in that same call, so leftovers from
+ *   an earlier call never leak into a result.
+ */
+int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D,
+                             int64_t row_stride, const float *gamma_q, const float *gamma_k,
+                             float eps, void *stream);
 
 /* Static English text for a qkn_status value (never NULL). */
 const char *qknorm_status_string(int status);

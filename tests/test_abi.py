@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
     assert set(names) == {"qknorm_per_head", "qknorm_layerwise", "qknorm_status_string",
                           "qknorm_last_cuda_error", "qknorm_version", "qknorm_layerwise_partials",
-                          "qknorm_layerwise_apply"}
+                          "qknorm_layerwise_apply", "qknorm_layerwise_noalloc"}
     for n in names:
         assert hasattr(lib, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", qbuild.LIB_PATH], capture_output=True,
@@ -133,6 +133,21 @@ def test_tensor_parallel_steps_validation(lib):
     assert app(P, *args, S, 4096, 1024, -1.0, None) == EPS
     assert app(P, BF16, 4, 32, 8, 128, W, None, G2, S, 4096, 1024, 1e-6, None) == NULL
     assert app(None, BF16, 0, 32, 8, 128, W, None, None, None, 4096, 1024, 1e-6, None) == OK
+    assert lib.qknorm_last_cuda_error() == 0
+
+
+def test_noalloc_validation(lib):
+    f = lib.qknorm_layerwise_noalloc
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                  ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    W = (32 + 16) * 128
+    assert f(P, BF16, 65537, 32, 8, 128, W, G1, G2, 1e-6, None) == -8  # beyond the scratch
+    assert lib.qknorm_status_string(-8).decode().startswith("T exceeds")
+    assert f(None, BF16, 4, 32, 8, 128, W, G1, G2, 1e-6, None) == NULL
+    assert f(P + 8, BF16, 4, 32, 8, 128, W, G1, G2, 1e-6, None) == ALIGN
+    assert f(None, BF16, 0, 32, 8, 128, W, None, None, 1e-6, None) == OK
     assert lib.qknorm_last_cuda_error() == 0
 
 
