@@ -21,5 +21,6 @@ from ._binding import (  # noqa: F401
     tp_allreduce_,
     tp_full_lengths,
     status_string,
+    wait_timeouts,
 )
 from .buildlib import LIB_PATH, build  # noqa: F401

@@ -17,6 +17,7 @@ QKN_BF16, QKN_FP32, QKN_FP16, QKN_FP8_E4M3 = 0, 1, 2, 3
 STATUS = {
     0: "QKN_OK", -1: "QKN_ERR_NULL", -2: "QKN_ERR_SHAPE", -3: "QKN_ERR_ALIGN",
     -4: "QKN_ERR_NSHARDS", -5: "QKN_ERR_UNSUPPORTED", -6: "QKN_ERR_CUDA", -7: "QKN_ERR_EPS",
+    -8: "QKN_ERR_TOO_LARGE",
 }
 
 _lock = threading.Lock()
@@ -60,6 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.qknorm_last_cuda_error.restype = i32
         lib.qknorm_version.argtypes = []
         lib.qknorm_version.restype = i32
+        lib.qknorm_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        lib.qknorm_wait_timeouts.restype = i32
         if path == LIB_PATH:
             _lib = lib
         return lib
@@ -118,6 +121,13 @@ def _device_check(qkv, *others):
     for g in others:
         if g is not None and g.device != qkv.device:
             raise ValueError("gamma and sums must live on the same device as qkv")
+
+
+def wait_timeouts() -> int:
+    """In-kernel waits on the current device that gave up (qknorm_wait_timeouts)."""
+    count = ctypes.c_uint(0)
+    _check("qknorm_wait_timeouts", load_library().qknorm_wait_timeouts(ctypes.byref(count)))
+    return int(count.value)
 
 
 def qknorm_per_head(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, row_stride=None, stream=None):

@@ -340,32 +340,114 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
 // --------------------------------------------------------------- layerwise --
 constexpr int kLayerwiseStages = 2;
 
-// Sum of squares of one vector of `nh` heads from their partials
-// part[0..nh), computed by one whole warp; every lane returns the same value.
+// How warp_sumsq reduces the nh head partials of one vector (q or k).  The
+// host fills it once per launch, so the token loop divides nothing.
+//   used:      lanes that hold partials, min(p, 32) with p the largest power
+//              of two dividing nh (0 when nh == 0);
+//   per_lane:  heads each of those lanes sums, in order (nh / used);
+//   per_shard: lanes per emulated shard (used / nshards).
+struct SumPlan {
+    int used;
+    int per_lane;
+    int per_shard;
+};
+
+// Sum of squares of one vector from its head partials part[0..nh), computed
+// by one whole warp; every lane returns the same value.
 //
-// The reduction tree is fixed by nh alone.  Let p be the largest power of two
-// dividing nh and u = min(p, 32) the lanes used: lane i sums heads
-// [i*c, (i+1)*c) in order (c = nh/u), then xor butterflies join lanes at
+// The reduction tree is fixed by nh alone: lane i sums heads
+// [i*per_lane, (i+1)*per_lane) in order, then xor butterflies join lanes at
 // distance 1, 2, 4, ...  With n shards (n a power of two dividing nh, so
-// n <= u), shard r holds exactly lanes [r*u/n, (r+1)*u/n): the butterflies
-// below distance u/n form each shard's partial S_r from that shard's heads
-// only, and the remaining ones are the scalar combine of S_0..S_{n-1}.  So
-// the result does not depend on n, bit for bit.
-__device__ __forceinline__ float warp_sumsq(const float *part, int nh, int nshards, int lane)
+// n <= used), shard r holds exactly lanes [r*used/n, (r+1)*used/n): the
+// butterflies below distance used/n form each shard's partial S_r from that
+// shard's heads only, and the remaining ones are the scalar combine of
+// S_0..S_{n-1}.  So the result does not depend on n, bit for bit.
+__device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p, int lane)
 {
-    if (nh == 0) return 0.f;
-    const int p2 = nh & (-nh);
-    const int used = p2 < 32 ? p2 : 32;
-    const int c = nh / used;
     float v = 0.f;
-    if (lane < used)
-        for (int j = 0; j < c; ++j) v += part[lane * c + j];
-    const int per_shard = used / nshards;
-    for (int o = 1; o < per_shard; o <<= 1)  // rank-local partial S_r
+    if (lane < p.used)
+        for (int j = 0; j < p.per_lane; ++j) v += part[lane * p.per_lane + j];
+    for (int o = 1; o < p.per_shard; o <<= 1)  // rank-local partial S_r
         v += __shfl_xor_sync(0xffffffffu, v, o);
-    for (int o = per_shard; o < used; o <<= 1)  // combine of the shard scalars
+    for (int o = p.per_shard; o < p.used; o <<= 1)  // combine of the shard scalars
         v += __shfl_xor_sync(0xffffffffu, v, o);
     return __shfl_sync(0xffffffffu, v, 0);
+}
+
+// ---- cluster exchange of head partials (transaction barriers) --
+// Each block of a cluster keeps two mbarriers, one per partials buffer.  The
+// owner of a head pushes that head's fp32 partial into the buffer of every
+// block of the cluster with st.async, which also counts its 4 bytes against
+// the receiving block's barrier; a block's barrier phase completes once all
+// (Hq + Hk) partials of the token have landed and its own thread 0 has armed
+// the phase.  No cluster-wide barrier and no memory fence is on the token path.
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(arrivals)
+                 : "memory");
+}
+// Make the initialised barriers visible to the other blocks of the cluster.
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// One arrival plus `bytes` expected transaction bytes for the current phase.
+__device__ __forceinline__ void mbar_arm(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// The shared::cluster address of `cta_addr` (a shared::cta address) in the
+// block of cluster rank `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t cta_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(cta_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_async_f32(uint32_t dst, float v, uint32_t bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                     dst),
+                 "r"(__float_as_uint(v)), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits on a barrier give up after this long (they complete in microseconds
+// when the exchange works); each give-up is counted in g_wait_timeouts.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ unsigned int g_wait_timeouts;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
 }
 
 // What a layerwise launch does with a token.
@@ -375,23 +457,27 @@ __device__ __forceinline__ float warp_sumsq(const float *part, int nh, int nshar
 //   kApply:    only the scaling, by 1/sqrt(aux[2t]/len_q + eps) for q and
 //              1/sqrt(aux[2t+1]/len_k + eps) for k, where aux holds the sums
 //              over all ranks and len_q, len_k the full vector lengths.
+// The mean S/L is formed as S * inv_len with inv_len = 1/L rounded to fp32
+// once per launch.
 enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 
 // A token's heads are split over the CL blocks of a thread-block cluster
 // (CL = 1 for a plain launch): block c of a cluster owns heads
 // [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
 // thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
-// per head).  Dynamic shared memory per block: kLayerwiseStages stages of
-// this block's part of a token (hc*D*sizeof(TS) bytes), then two buffers of
-// `heads` fp32 head partials (alternating per token).  With CL > 1 every block
-// writes its head partials into all blocks of its cluster (distributed shared
-// memory) before the cluster barrier, so each block then holds all of them.
+// per head), and thread l == 0 is the head's owner.  Dynamic shared memory
+// per block: kLayerwiseStages stages of this block's part of a token
+// (hc*D*sizeof(TS) bytes), two buffers of `heads` fp32 head partials
+// (alternating per token), then the two exchange barriers (CL > 1).  With
+// CL = 1 the partials meet behind one block barrier per token; with CL > 1
+// each owner pushes its partial into every block of the cluster and each
+// block waits on its own barrier (see the exchange helpers above).
 template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode>
 __global__ void __launch_bounds__(1024)
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
-                     int nshards, const float *__restrict__ gamma_q,
-                     const float *__restrict__ gamma_k, float eps, float len_q, float len_k,
-                     float *__restrict__ aux)
+                     const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
+                     float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                     SumPlan plan_k, float *__restrict__ aux)
 {
     using S = Storage<TS>;
     using V = typename S::Vec;
@@ -401,6 +487,7 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     constexpr int kLPH = kNV / VPT;   // threads per head
     constexpr int kEPT = VPT * kVec;  // elements per thread
     constexpr int NST = kLayerwiseStages;
+    constexpr bool kExchange = kCluster && kMode != kApply;
     static_assert(kNV % VPT == 0 && 32 % kLPH == 0, "head must map onto a sub-warp");
 
     extern __shared__ __align__(16) unsigned char smem[];
@@ -414,6 +501,8 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     const int h_lo = crank * hc;
     const int span = hc * D * (int)sizeof(TS);
     float *part = reinterpret_cast<float *>(smem + (size_t)NST * span);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(part + 2 * heads);
+    const uint32_t token_bytes = (uint32_t)heads * (uint32_t)sizeof(float);
     const int hl = threadIdx.x / kLPH;   // head within this block
     const int h = h_lo + hl;
     const int l = threadIdx.x % kLPH;
@@ -457,13 +546,23 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     };
 #pragma unroll
     for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
-    // Distributed shared memory may only be touched once every block of the
-    // cluster is running: meet once before the first remote write.  (The last
-    // remote write of the loop precedes its final cluster barrier, so no block
-    // exits while another may still write into it.)
-    if constexpr (kCluster && kMode != kApply) cooperative_groups::this_cluster().sync();
-    int st = 0, pb = 0;
-    for (int64_t t = first; t < T; t += stride) {
+    if constexpr (kExchange) {
+        if (threadIdx.x == 0) {
+            mbar_init(&bar[0], 1);
+            mbar_init(&bar[1], 1);
+            mbar_init_fence();
+            mbar_arm(&bar[0], token_bytes);
+            mbar_arm(&bar[1], token_bytes);
+        }
+        // Distributed shared memory may only be touched once every block of
+        // the cluster is running: meet once, barriers initialised and armed,
+        // before the first remote write.
+        cooperative_groups::this_cluster().sync();
+    }
+    int st = 0;
+    uint32_t it = 0;  // tokens this block has done; partials buffer it % 2
+    bool timed_out = false;
+    for (int64_t t = first; t < T; t += stride, ++it) {
         // Refill the stage this thread finished with on the previous token.
         fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
         cp_async_wait<NST - 1>();
@@ -471,27 +570,42 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         float rq = 0.f, rk = 0.f;
         if constexpr (kMode == kApply) {
             // Sums over all ranks come in; no exchange inside the launch.
-            if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) / len_q + eps);
-            if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) / len_k + eps);
+            if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) * inv_len_q + eps);
+            if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) * inv_len_k + eps);
         } else {
             float s = 0.f;
-    #pragma unroll
+#pragma unroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec];
                 S::unpack(active ? sp[l + v * kLPH] : zero_vec<V>(), f);
-    #pragma unroll
+#pragma unroll
                 for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
             }
             s = group_sum<kLPH>(s);
-            // Partials alternate between two buffers: a warp still reading this
-            // token's buffer cannot meet a write of the next token's, which only
-            // starts after the next barrier (of the block, or of the cluster).
+            // Partials alternate between two buffers.  The next write into
+            // this token's buffer is for the token after next; every block
+            // sends it only after the token in between, which needs a partial
+            // from every warp of the cluster, and each warp sends that only
+            // after it has finished reading this buffer.  (Every warp holds an
+            // owner: its first thread.)
+            const uint32_t pb = it & 1u;
             float *pp = part + pb * heads;
-            if constexpr (kCluster) {
-                cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
-                if (active && l == 0)
-                    for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(pp + h, r) = s;
-                cluster.sync();
+            if constexpr (kExchange) {
+                if (active && l == 0) {
+                    const uint32_t dst = smem_u32(pp + h), b = smem_u32(&bar[pb]);
+                    for (int r = 0; r < cl; ++r)
+                        st_async_f32(cluster_addr(dst, (uint32_t)r), s,
+                                     cluster_addr(b, (uint32_t)r));
+                }
+                // Buffer pb serves every other token: phase it/2 of its barrier.
+                if (!timed_out && !mbar_wait_bounded(&bar[pb], (it >> 1) & 1u)) {
+                    timed_out = true;
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
+                }
+                // Arm the barrier's next phase (the token after next) before this
+                // thread sends its next partial, which any sender of that phase
+                // has to wait for.
+                if (threadIdx.x == 0 && !timed_out) mbar_arm(&bar[pb], token_bytes);
             } else {
                 if (active && l == 0) pp[h] = s;
                 __syncthreads();
@@ -499,16 +613,16 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
             if constexpr (kMode == kPartials) {
                 // One warp of the cluster's first block writes this rank's sums.
                 if (threadIdx.x < 32 && crank == 0) {
-                    const float sq = warp_sumsq(pp, Hq, 1, lane);
-                    const float sk = warp_sumsq(pp + Hq, Hk, 1, lane);
+                    const float sq = warp_sumsq(pp, plan_q, lane);
+                    const float sk = warp_sumsq(pp + Hq, plan_k, lane);
                     if (lane == 0) {
                         aux[2 * t] = sq;
                         aux[2 * t + 1] = sk;
                     }
                 }
             } else {
-                if (need_q) rq = rsqrtf(warp_sumsq(pp, Hq, nshards, lane) / len_q + eps);
-                if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, Hk, nshards, lane) / len_k + eps);
+                if (need_q) rq = rsqrtf(warp_sumsq(pp, plan_q, lane) * inv_len_q + eps);
+                if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, plan_k, lane) * inv_len_k + eps);
             }
         }
         if (kMode != kPartials && active) {
@@ -530,9 +644,10 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
             }
         }
         st = (st + 1 == NST) ? 0 : st + 1;
-        pb ^= 1;
     }
     cp_async_wait<0>();
+    // No block leaves while a partner could still write into it.
+    if constexpr (kExchange) cooperative_groups::this_cluster().sync();
 }
 
 // ------------------------------------------------------------------- host --
@@ -722,15 +837,17 @@ constexpr bool layerwise_gamma_regs()
 
 template <typename TS, int D, int VPT, bool kCluster, int kMode>
 int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
-                         const float *gq, const float *gk, float eps, int nshards, int threads,
-                         int cluster, float len_q, float len_k, float *aux, cudaStream_t stream)
+                         const float *gq, const float *gk, float eps, int threads, int cluster,
+                         float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
+                         float *aux, cudaStream_t stream)
 {
     auto kern =
         qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>(), kCluster, kMode>;
     static KernelCache kc;
     const int heads = Hq + Hk;
     const size_t span = (size_t)(heads / cluster) * D * sizeof(TS);
-    const size_t smem = kLayerwiseStages * span + (size_t)2 * heads * sizeof(float);
+    const size_t smem =
+        kLayerwiseStages * span + (size_t)2 * heads * sizeof(float) + 2 * sizeof(uint64_t);
     int dev = 0, rc;
     DeviceInfo info;
     if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
@@ -766,8 +883,8 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
     if (cap < 1) return QKN_ERR_UNSUPPORTED;
     const int64_t clusters = T < cap ? T : cap;
     return launch_pdl(kern, (unsigned)(clusters * cluster), threads, smem, stream,
-                      (unsigned)cluster, static_cast<TS *>(qkv), row_stride, T, Hq, Hk, nshards,
-                      gq, gk, eps, len_q, len_k, aux);
+                      (unsigned)cluster, static_cast<TS *>(qkv), row_stride, T, Hq, Hk, gq, gk,
+                      eps, inv_len_q, inv_len_k, plan_q, plan_k, aux);
 }
 
 // Launch shape.  First choice: the smallest cluster (1, 2, 4 or 8 blocks,
@@ -778,6 +895,19 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 constexpr int kLayerwiseTargetThreads = 256;
 constexpr int kMaxCluster = 8;
 
+// The reduction plan of warp_sumsq for nh head partials split into nshards.
+SumPlan sum_plan(int nh, int nshards)
+{
+    SumPlan p = {0, 0, 0};
+    if (nh > 0) {
+        const int p2 = nh & (-nh);
+        p.used = p2 < 32 ? p2 : 32;
+        p.per_lane = nh / p.used;
+        p.per_shard = p.used / nshards;  // nshards is a power of two dividing nh
+    }
+    return p;
+}
+
 // len_q, len_k: the normalised lengths (the full vectors; for kFused and
 // kPartials they are this launch's own Hq*D and Hk*D).
 template <typename TS, int D, int kMode = kFused>
@@ -787,6 +917,9 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
 {
     if (len_q < 0.f) len_q = (float)((int64_t)Hq * D);  // exact: spans are < 2^24 elements
     if (len_k < 0.f) len_k = (float)((int64_t)Hk * D);
+    const float inv_len_q = Hq > 0 ? 1.0f / len_q : 0.f;
+    const float inv_len_k = Hk > 0 ? 1.0f / len_k : 0.f;
+    const SumPlan plan_q = sum_plan(Hq, nshards), plan_k = sum_plan(Hk, nshards);
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kVec = Storage<TS>::kVec;
     const int64_t heads = Hq + Hk;
@@ -820,12 +953,12 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
             if constexpr (layerwise_gamma_regs<TS, V>()) {                                     \
                 if (cluster > 1)                                                               \
                     return launch_layerwise_vpt<TS, D, V, true, kMode>(                        \
-                        qkv, T, Hq, Hk, row_stride, gq, gk, eps, nshards, threads, cluster,    \
-                        len_q, len_k, aux, stream);                                            \
+                        qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, cluster, inv_len_q,  \
+                        inv_len_k, plan_q, plan_k, aux, stream);                               \
             }                                                                                  \
             return launch_layerwise_vpt<TS, D, V, false, kMode>(                               \
-                qkv, T, Hq, Hk, row_stride, gq, gk, eps, nshards, threads, 1, len_q, len_k,    \
-                aux, stream);                                                                  \
+                qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, 1, inv_len_q, inv_len_k,     \
+                plan_q, plan_k, aux, stream);                                                  \
         }                                                                                      \
         break;
     switch (chosen) {
@@ -1018,6 +1151,13 @@ const char *qknorm_status_string(int status)
 
 int qknorm_last_cuda_error(void) { return g_last_cuda_error; }
 
-int qknorm_version(void) { return 102; }
+int qknorm_wait_timeouts(unsigned int *count)
+{
+    if (count == nullptr) return QKN_ERR_NULL;
+    const cudaError_t e = cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned int));
+    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
+}
+
+int qknorm_version(void) { return 103; }
 
 }  // extern "C"

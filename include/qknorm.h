@@ -17,9 +17,10 @@
  *
  * Arithmetic: elements are widened to fp32, sums of squares accumulate in
  * fp32, the inverse RMS is 1/sqrt(S/L + eps) in fp32 (L = normalised length,
- * eps inside the square root), and each output x * rinv * gamma is rounded
- * once to the storage type: round to nearest even for bf16 and fp16, and for
- * FP8 E4M3 round to nearest even saturating to +-448.
+ * eps inside the square root; S/L is formed as S times 1/L rounded to fp32),
+ * and each output x * rinv * gamma is rounded once to the storage type:
+ * round to nearest even for bf16 and fp16, and for FP8 E4M3 round to nearest
+ * even saturating to +-448.
  *
  * Common arguments
  *   qkv         device pointer to the fused buffer; 16-byte aligned.
@@ -109,9 +110,14 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
  * is bit-identical for every valid nshards.  A token's heads are split over
  * a thread-block cluster of 1, 2, 4 or 8 blocks (C, which must divide
  * Hq + Hk); each block keeps two tokens' worth of its heads staged in shared
- * memory, so 2 * (Hq + Hk) / C * D * sizeof(element) + 8 * (Hq + Hk) bytes
- * must fit the device's opt-in shared memory per block (227 KiB on B200) for
- * the cluster size chosen, else QKN_ERR_UNSUPPORTED.
+ * memory, so 2 * (Hq + Hk) / C * D * sizeof(element) + 8 * (Hq + Hk) + 16
+ * bytes must fit the device's opt-in shared memory per block (227 KiB on
+ * B200) for the cluster size chosen, else QKN_ERR_UNSUPPORTED.  The blocks of
+ * a cluster pass head partials to one another through distributed shared
+ * memory and wait for them on transaction barriers; each such wait gives up
+ * after 2 seconds, which can only happen if the GPU misbehaves, and is then
+ * counted (see qknorm_wait_timeouts) while the kernel runs to its end with
+ * wrong results.
  */
 int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
                      const float *gamma_q, const float *gamma_k, float eps, int nshards,
@@ -186,8 +192,15 @@ const char *qknorm_status_string(int status);
 /* cudaError_t of the calling thread's last QKN_ERR_CUDA (0 if none). */
 int qknorm_last_cuda_error(void);
 
+/* Number of in-kernel waits on the current device that gave up since the
+ * library was loaded (see qknorm_layerwise); 0 in correct operation.  Copies
+ * one device counter to *count with a blocking copy on the legacy default
+ * stream, so the work queued before it has finished.  QKN_ERR_NULL if count
+ * is NULL, QKN_ERR_CUDA if the copy fails. */
+int qknorm_wait_timeouts(unsigned int *count);
+
 /* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3, 1.02 the
- * tensor-parallel layerwise steps). */
+ * tensor-parallel layerwise steps, 1.03 qknorm_wait_timeouts). */
 int qknorm_version(void);
 
 #ifdef __cplusplus

@@ -38,7 +38,8 @@ def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
     assert set(names) == {"qknorm_per_head", "qknorm_layerwise", "qknorm_status_string",
                           "qknorm_last_cuda_error", "qknorm_version", "qknorm_layerwise_partials",
-                          "qknorm_layerwise_apply", "qknorm_layerwise_noalloc"}
+                          "qknorm_layerwise_apply", "qknorm_layerwise_noalloc",
+                          "qknorm_wait_timeouts"}
     for n in names:
         assert hasattr(lib, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", qbuild.LIB_PATH], capture_output=True,
@@ -48,12 +49,14 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.qknorm_version() == 102
-    for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS):
+    assert lib.qknorm_version() == 103
+    for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS, -8):
         s = lib.qknorm_status_string(code).decode()
         assert s and s != "unknown status"
     assert lib.qknorm_status_string(42).decode() == "unknown status"
     assert lib.qknorm_last_cuda_error() == 0
+    # Only the argument check runs without a GPU.
+    assert lib.qknorm_wait_timeouts(None) == NULL
 
 
 def ph(lib, qkv=P, dtype=BF16, T=4, Hq=16, Hk=2, D=128, stride=None, gq=G1, gk=G2, eps=1e-6):

@@ -324,3 +324,10 @@ def test_tensor_parallel_partials_leave_buffer_untouched():
     want = np.stack([(x[:, :4096] ** 2).sum(1), (x[:, 4096:5120] ** 2).sum(1)], 1)
     got = part.cpu().numpy().astype(np.float64)
     assert np.allclose(got, want, rtol=1e-5, atol=0)
+
+
+def test_no_in_kernel_wait_gave_up():
+    """The cluster exchange waits of every launch above completed: none ran into
+    its time limit (which would have left wrong results behind)."""
+    torch.cuda.synchronize()
+    assert qkn.wait_timeouts() == 0
