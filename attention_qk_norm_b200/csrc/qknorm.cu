@@ -473,11 +473,11 @@ enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 // each owner pushes its partial into every block of the cluster and each
 // block waits on its own barrier (see the exchange helpers above).
 template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode>
-__global__ void __launch_bounds__(1024)
-qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
-                     const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
-                     float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
-                     SumPlan plan_k, float *__restrict__ aux)
+__device__ __forceinline__ void
+layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                 const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
+                 float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
+                 float *__restrict__ aux)
 {
     using S = Storage<TS>;
     using V = typename S::Vec;
@@ -488,6 +488,9 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     constexpr int kEPT = VPT * kVec;  // elements per thread
     constexpr int NST = kLayerwiseStages;
     constexpr bool kExchange = kCluster && kMode != kApply;
+    // Vector loops unroll fully when gamma sits in registers (indexed by v);
+    // with gamma in L1 the long loops unroll by 8.
+    constexpr int kUnroll = kGammaRegs || VPT < 8 ? VPT : 8;
     static_assert(kNV % VPT == 0 && 32 % kLPH == 0, "head must map onto a sub-warp");
 
     extern __shared__ __align__(16) unsigned char smem[];
@@ -531,16 +534,15 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
             for (int e = 0; e < kVec; ++e) g[v * kVec + e] = t4[e];
         }
     }
-    const int64_t col0 = (int64_t)h * D;              // in the token row
-    const size_t scol0 = (size_t)hl * D * sizeof(TS);  // in a stage
+    const int64_t col0 = (int64_t)h * D;          // in the token row
+    const int scol0 = (hl * D + l * kVec) * (int)sizeof(TS);  // in a stage
     // Each thread copies, and later reads, only its own vectors of a stage.
     auto fetch = [&](int64_t tok, int st) {
         if (active && tok < T) {
             const V *src = reinterpret_cast<const V *>(qkv + tok * row_stride + col0);
-            unsigned char *dst = smem + (size_t)st * span + scol0;
-#pragma unroll
-            for (int v = 0; v < VPT; ++v)
-                cp_async<kVB>(dst + (l + v * kLPH) * kVB, src + l + v * kLPH);
+            V *dst = reinterpret_cast<V *>(smem + (size_t)st * span + scol0);
+#pragma unroll kUnroll
+            for (int v = 0; v < VPT; ++v) cp_async<kVB>(dst + v * kLPH, src + l + v * kLPH);
         }
         cp_async_commit();
     };
@@ -574,10 +576,10 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
             if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) * inv_len_k + eps);
         } else {
             float s = 0.f;
-#pragma unroll
+#pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec];
-                S::unpack(active ? sp[l + v * kLPH] : zero_vec<V>(), f);
+                S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
 #pragma unroll
                 for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
             }
@@ -628,10 +630,10 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
         if (kMode != kPartials && active) {
             const float rinv = h < Hq ? rq : rk;
             V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
-#pragma unroll
+#pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec], o[kVec], gv[kVec];
-                S::unpack(sp[l + v * kLPH], f);
+                S::unpack(sp[v * kLPH], f);
                 if constexpr (kGammaRegs) {
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
@@ -648,6 +650,54 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     cp_async_wait<0>();
     // No block leaves while a partner could still write into it.
     if constexpr (kExchange) cooperative_groups::this_cluster().sync();
+}
+
+// Registers per thread: 40, 48 or 56 when a thread keeps 8, 16 or 32
+// elements (and as many gamma values) per token.  The caps fit without
+// spilling and leave room for more resident blocks than the compiler's own
+// choice (up to 64); measured on B200 they are the fastest for every storage
+// type and head_dim.
+#ifndef QKN_LW_REGS8
+#define QKN_LW_REGS8 40
+#endif
+#ifndef QKN_LW_REGS16
+#define QKN_LW_REGS16 48
+#endif
+#ifndef QKN_LW_REGS32
+#define QKN_LW_REGS32 56
+#endif
+template <typename TS, int VPT>
+constexpr int layerwise_max_regs()
+{
+    constexpr int kEPT = VPT * Storage<TS>::kVec;
+    return kEPT <= 8 ? QKN_LW_REGS8 : (kEPT <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32);
+}
+
+// Gamma in registers (at most 32 elements per thread).
+template <typename TS, int D, int VPT, bool kCluster, int kMode>
+__global__ void __maxnreg__((layerwise_max_regs<TS, VPT>()))
+qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                     const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
+                     float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                     SumPlan plan_k, float *__restrict__ aux)
+{
+    layerwise_tokens<TS, D, VPT, true, kCluster, kMode>(qkv, row_stride, T, Hq, Hk, gamma_q,
+                                                        gamma_k, eps, inv_len_q, inv_len_k,
+                                                        plan_q, plan_k, aux);
+}
+
+// Gamma read through L1 (tokens too wide for registers; one block per token,
+// up to 1024 threads).
+template <typename TS, int D, int VPT, int kMode>
+__global__ void __launch_bounds__(1024)
+qkn_layerwise_l1_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                        const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
+                        float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                        SumPlan plan_k, float *__restrict__ aux)
+{
+    layerwise_tokens<TS, D, VPT, false, false, kMode>(qkv, row_stride, T, Hq, Hk, gamma_q,
+                                                      gamma_k, eps, inv_len_q, inv_len_k, plan_q,
+                                                      plan_k, aux);
 }
 
 // ------------------------------------------------------------------- host --
@@ -841,8 +891,12 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
                          float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
                          float *aux, cudaStream_t stream)
 {
-    auto kern =
-        qkn_layerwise_kernel<TS, D, VPT, layerwise_gamma_regs<TS, VPT>(), kCluster, kMode>;
+    auto kern = [] {
+        if constexpr (layerwise_gamma_regs<TS, VPT>())
+            return qkn_layerwise_kernel<TS, D, VPT, kCluster, kMode>;
+        else
+            return qkn_layerwise_l1_kernel<TS, D, VPT, kMode>;
+    }();
     static KernelCache kc;
     const int heads = Hq + Hk;
     const size_t span = (size_t)(heads / cluster) * D * sizeof(TS);
@@ -887,13 +941,38 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
                       eps, inv_len_q, inv_len_k, plan_q, plan_k, aux);
 }
 
-// Launch shape.  First choice: the smallest cluster (1, 2, 4 or 8 blocks,
-// dividing the head count) and the fewest vectors per thread that keep gamma
-// in registers and the block within 256 threads.  Otherwise one block per
-// token, the fewest vectors per thread within 256 threads, else 1024, with
-// gamma read through L1 where it does not fit registers.
-constexpr int kLayerwiseTargetThreads = 256;
+// Launch shape, chosen from measurements on B200 over the four storage types,
+// head_dim 64 to 256 and 40 to 72 heads:
+//  * the smallest cluster size CL (1, 2, 4 or 8 blocks, dividing the head
+//    count) for which some vectors-per-thread count VPT keeps gamma in
+//    registers (VPT * kVec <= 32) and the block within 576 threads;
+//  * the fewest such VPT, but at least 2: with one vector per thread the
+//    per-token work of a thread is too short for its fixed per-token cost;
+//  * on short inputs, fewer than 12 tokens per resident cluster, twice that
+//    VPT when gamma still fits: half the threads per block, about twice the
+//    resident blocks, so more tokens are under way at once.
+// If no cluster size fits, one block per token with the fewest VPT within
+// 1024 threads, gamma read through L1 where it does not fit registers.
+constexpr int kLayerwiseMaxThreads = 576;
+constexpr int kLayerwiseShortTokens = 12;
 constexpr int kMaxCluster = 8;
+
+// Registers per thread of the gamma-in-registers kernel for `ept` elements
+// per thread (layerwise_max_regs at run time).
+int layerwise_regs(int ept)
+{
+    return ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32);
+}
+
+// Resident blocks per SM by the register file and the thread limit; the
+// shape rule's estimate (the launch itself queries the occupancy).
+int layerwise_blocks_estimate(int threads, int regs)
+{
+    const int by_regs = 65536 / (threads * ((regs + 7) / 8 * 8));
+    const int by_threads = 2048 / threads;
+    const int n = by_regs < by_threads ? by_regs : by_threads;
+    return n < 32 ? n : 32;
+}
 
 // The reduction plan of warp_sumsq for nh head partials split into nshards.
 SumPlan sum_plan(int nh, int nshards)
@@ -923,28 +1002,32 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kVec = Storage<TS>::kVec;
     const int64_t heads = Hq + Hk;
+    auto vpt_ok = [](int vpt) { return vpt <= kNV && kNV % vpt == 0 && kNV / vpt <= 32; };
+    auto threads_for = [&](int cl, int vpt) {
+        return (int)(((heads / cl * (kNV / vpt)) + 31) / 32 * 32);
+    };
     int chosen = 0, cluster = 1;
     for (int cl = 1; cl <= kMaxCluster && chosen == 0; cl *= 2) {
         if (heads % cl != 0) continue;
-        for (int vpt = 1; vpt <= kNV && vpt * kVec <= 32; vpt *= 2) {
-            if (kNV % vpt != 0 || kNV / vpt > 32) continue;  // mirrors layerwise_vpt_ok
-            if (((heads / cl * (kNV / vpt) + 31) / 32) * 32 <= kLayerwiseTargetThreads) {
+        for (int vpt = 2; vpt * kVec <= 32; vpt *= 2) {
+            if (vpt_ok(vpt) && threads_for(cl, vpt) <= kLayerwiseMaxThreads) {
                 chosen = vpt;
                 cluster = cl;
                 break;
             }
         }
     }
-    for (int pass = 0; pass < 2 && chosen == 0; ++pass) {
-        const int64_t limit = pass == 0 ? kLayerwiseTargetThreads : 1024;
-        for (int vpt = 1; vpt <= kNV; vpt *= 2) {
-            if (kNV % vpt != 0 || kNV / vpt > 32) continue;
-            if (((heads * (kNV / vpt) + 31) / 32) * 32 <= limit) {
-                chosen = vpt;
-                break;
-            }
-        }
+    if (chosen != 0 && 2 * chosen * kVec <= 32 && vpt_ok(2 * chosen)) {
+        int dev = 0, rc;
+        DeviceInfo info;
+        if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
+        const int per_sm = layerwise_blocks_estimate(threads_for(cluster, chosen),
+                                                     layerwise_regs(chosen * kVec));
+        const int64_t pipelines = (int64_t)info.sms * per_sm / cluster;  // resident clusters
+        if (T < kLayerwiseShortTokens * pipelines) chosen *= 2;
     }
+    for (int vpt = 1; vpt <= kNV && chosen == 0; vpt *= 2)
+        if (vpt_ok(vpt) && threads_for(1, vpt) <= 1024) chosen = vpt;
     if (chosen == 0) return QKN_ERR_UNSUPPORTED;
     const int threads = (int)(((heads / cluster * (kNV / chosen)) + 31) / 32 * 32);
 #define QKN_LW_CASE(V)                                                                         \

@@ -179,9 +179,9 @@ def test_layerwise_head_counts(Hq, Hk, ns):
 @pytest.mark.parametrize("D", synth.STRESS_D)
 @pytest.mark.parametrize("Hq,Hk,ns", [(64, 8, (1, 8)), (32, 4, (1, 4)), (30, 5, (1, 5))])
 def test_layerwise_wide_tokens(dtype, D, Hq, Hk, ns):
-    """Wide tokens: heads split over a thread-block cluster (72 or 36 heads),
-    or one block with gamma read through L1 (35 heads: no cluster size
-    divides the head count)."""
+    """Wide tokens: one block of up to 576 threads, or heads split over a
+    thread-block cluster where a block would need more (72 or 36 heads at
+    head_dim 256), or an odd head count (35) that no cluster size divides."""
     ns = tuple(n for n in ns if n in (1, 2, 4, 8))
     c = synth.make_case(45, Hq, Hk, D, dtype=dtype, seed=Hq + D, layerwise=True, scale="stress",
                         zero_frac=0.05, outlier_frac=0.05)
@@ -189,6 +189,15 @@ def test_layerwise_wide_tokens(dtype, D, Hq, Hk, ns):
             for n in ns]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
+
+
+@pytest.mark.parametrize("dtype", (synth.BF16, synth.FP8))
+def test_layerwise_gamma_through_l1(dtype):
+    """129 heads of 256 (odd, so no cluster split): gamma cannot stay in
+    registers within 1024 threads, so the kernel reads it through L1."""
+    c = synth.make_case(37, 121, 8, 256, dtype=dtype, seed=61, layerwise=True, scale="stress",
+                        zero_frac=0.05, outlier_frac=0.05)
+    full_parity(c, "layerwise", 1, what="gamma through L1 %s" % dtype)
 
 
 @pytest.mark.parametrize("dtype", (synth.FP16, synth.FP8))
