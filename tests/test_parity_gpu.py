@@ -191,6 +191,28 @@ def test_layerwise_wide_tokens(dtype, D, Hq, Hk, ns):
         assert np.array_equal(o, outs[0])
 
 
+@pytest.mark.parametrize("Hq,Hk,D,dtype,ns", [
+    (112, 16, 256, synth.BF16, (1, 2, 8)),  # 2-block clusters of 512 threads
+    (144, 16, 256, synth.FP16, (1, 8)),     # 4-block clusters
+    (256, 64, 256, synth.BF16, (1, 4)),     # 8-block clusters
+    (64, 16, 256, synth.FP32, (1, 8)),      # 2-block clusters, fp32
+    (112, 16, 256, synth.FP8, (1, 4)),      # 2-block clusters, FP8
+])
+def test_layerwise_cluster_split(Hq, Hk, D, dtype, ns):
+    """Tokens too wide for one block of 576 threads with gamma in registers:
+    the heads are split over a cluster of 2, 4 or 8 blocks, which pass head
+    partials to one another through distributed shared memory.  700 tokens
+    give every cluster several tokens, so both partials buffers and several
+    phases of their barriers are used.  Outputs are identical for every
+    nshards."""
+    c = synth.make_case(700, Hq, Hk, D, dtype=dtype, seed=Hq + Hk + D, layerwise=True,
+                        scale="stress", zero_frac=0.05, outlier_frac=0.05)
+    outs = [full_parity(c, "layerwise", n, what="cluster %s %d/%d n=%d" % (dtype, Hq, Hk, n))[0]
+            for n in ns]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
 @pytest.mark.parametrize("dtype", (synth.BF16, synth.FP8))
 def test_layerwise_gamma_through_l1(dtype):
     """129 heads of 256 (odd, so no cluster split): gamma cannot stay in
@@ -284,7 +306,8 @@ def _rank_columns(c, n, r):
 
 
 @pytest.mark.parametrize("Hq,Hk,D,dtype", [(32, 8, 128, synth.BF16), (64, 8, 256, synth.FP32),
-                                           (32, 8, 64, synth.FP8), (16, 8, 128, synth.FP16)])
+                                           (32, 8, 64, synth.FP8), (16, 8, 128, synth.FP16),
+                                           (112, 16, 256, synth.BF16)])
 @pytest.mark.parametrize("n", (1, 2, 4, 8))
 def test_tensor_parallel_steps_emulated(Hq, Hk, D, dtype, n):
     """n ranks emulated one after another on one GPU: each rank's partial sums,
