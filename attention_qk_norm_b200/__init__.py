@@ -17,7 +17,9 @@ from ._binding import (  # noqa: F401
     qknorm_layerwise_apply,
     qknorm_layerwise_partials,
     qknorm_layerwise_tp,
+    qknorm_layerwise_tp_allgather,
     qknorm_per_head,
+    tp_allgather_full,
     tp_allreduce_,
     tp_full_lengths,
     status_string,

@@ -212,6 +212,28 @@ def tp_full_lengths(Hq, Hk, D, world):
     return Hq * D * world, Hk * D * world
 
 
+def tp_allgather_full(xq, xk, group=None):
+    """All-gather this rank's q and k columns ([T, hq*D] and [T, hk*D]) over
+    ``group``; returns (full q [T, world*hq*D], full k [T, world*hk*D], world,
+    rank) with the ranks' columns in rank order.  Without an initialised
+    process group it returns the inputs themselves, world 1 and rank 0."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return xq, xk, 1, 0
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    if world == 1:
+        return xq, xk, 1, rank
+
+    def gather(x):
+        parts = [torch.empty_like(x) for _ in range(world)]
+        dist.all_gather(parts, x.contiguous(), group=group)
+        return torch.cat(parts, dim=1)
+
+    return gather(xq), gather(xk), world, rank
+
+
 def qknorm_layerwise_tp(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, group=None, row_stride=None):
     """Layerwise QK-Norm across a tensor-parallel group, in place.
 
@@ -225,3 +247,31 @@ def qknorm_layerwise_tp(qkv, Hq, Hk, D, gamma_q, gamma_k, eps, group=None, row_s
     len_q, len_k = tp_full_lengths(Hq, Hk, D, world)
     return qknorm_layerwise_apply(qkv, Hq, Hk, D, gamma_q, gamma_k, partials, len_q, len_k, eps,
                                   row_stride=row_stride)
+
+
+def qknorm_layerwise_tp_allgather(qkv, Hq, Hk, D, gamma_q_full, gamma_k_full, eps, group=None,
+                                  row_stride=None):
+    """The All-Gather baseline of tensor-parallel layerwise QK-Norm, in place:
+    the standard exchange that SwiftQK's scalar all-reduce replaces.  Every
+    rank of ``group`` gathers the q and k columns of all ranks (the full
+    vectors of every token, (world-1)*T*(Hq+Hk)*D elements received per rank
+    instead of 2*T scalars), normalises them with the full-length weights
+    ``gamma_q_full`` [world*Hq*D] and ``gamma_k_full`` [world*Hk*D] in
+    qknorm_layerwise, and keeps its own slice.  The result equals that of
+    qknorm_layerwise_tp up to the fp32 summation order."""
+    import torch
+
+    _device_check(qkv, gamma_q_full, gamma_k_full)
+    T, stride = _rows(qkv, row_stride)
+    q0, k0, k1 = 0, Hq * D, (Hq + Hk) * D
+    fq, fk, world, rank = tp_allgather_full(qkv[:, q0:k0], qkv[:, k0:k1], group)
+    HQ, HK = world * Hq, world * Hk
+    # A fused buffer of the full vectors; its V columns exist only to satisfy
+    # the layout and are never read.
+    full = torch.empty((T, (HQ + 2 * HK) * D), dtype=qkv.dtype, device=qkv.device)
+    full[:, :HQ * D] = fq
+    full[:, HQ * D:(HQ + HK) * D] = fk
+    qknorm_layerwise(full, HQ, HK, D, gamma_q_full, gamma_k_full, eps)
+    qkv[:, q0:k0] = full[:, rank * Hq * D:(rank + 1) * Hq * D]
+    qkv[:, k0:k1] = full[:, HQ * D + rank * Hk * D:HQ * D + (rank + 1) * Hk * D]
+    return qkv

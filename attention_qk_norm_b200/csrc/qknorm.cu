@@ -472,7 +472,7 @@ enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 // CL = 1 the partials meet behind one block barrier per token; with CL > 1
 // each owner pushes its partial into every block of the cluster and each
 // block waits on its own barrier (see the exchange helpers above).
-template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode>
+template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode, bool kOverlap>
 __device__ __forceinline__ void
 layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                  const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
@@ -570,6 +570,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
         cp_async_wait<NST - 1>();
         const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
         float rq = 0.f, rk = 0.f;
+        float xg[kOverlap ? kEPT : 1];  // x * gamma, formed before the combine
         if constexpr (kMode == kApply) {
             // Sums over all ranks come in; no exchange inside the launch.
             if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) * inv_len_q + eps);
@@ -582,6 +583,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
 #pragma unroll
                 for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
+                if constexpr (kOverlap) {
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) xg[v * kVec + e] = f[e] * g[v * kVec + e];
+                }
             }
             s = group_sum<kLPH>(s);
             // Partials alternate between two buffers.  The next write into
@@ -632,16 +637,22 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
             V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
 #pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
-                float f[kVec], o[kVec], gv[kVec];
-                S::unpack(sp[v * kLPH], f);
-                if constexpr (kGammaRegs) {
+                float o[kVec];
+                if constexpr (kOverlap) {
 #pragma unroll
-                    for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
+                    for (int e = 0; e < kVec; ++e) o[e] = xg[v * kVec + e] * rinv;
                 } else {
-                    load_gamma<kVec>(gb + (l + v * kLPH) * kVec, gv);
-                }
+                    float f[kVec], gv[kVec];
+                    S::unpack(sp[v * kLPH], f);
+                    if constexpr (kGammaRegs) {
 #pragma unroll
-                for (int e = 0; e < kVec; ++e) o[e] = f[e] * rinv * gv[e];
+                        for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
+                    } else {
+                        load_gamma<kVec>(gb + (l + v * kLPH) * kVec, gv);
+                    }
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) o[e] = f[e] * gv[e] * rinv;
+                }
                 store_stream(p + l + v * kLPH, S::pack(o));
             }
         }
@@ -656,7 +667,8 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 // elements (and as many gamma values) per token.  The caps fit without
 // spilling and leave room for more resident blocks than the compiler's own
 // choice (up to 64); measured on B200 they are the fastest for every storage
-// type and head_dim.
+// type and head_dim.  The overlap variant also keeps the thread's x * gamma
+// products across the combine: 48, 64 or 96.
 #ifndef QKN_LW_REGS8
 #define QKN_LW_REGS8 40
 #endif
@@ -666,24 +678,37 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #ifndef QKN_LW_REGS32
 #define QKN_LW_REGS32 56
 #endif
-template <typename TS, int VPT>
-constexpr int layerwise_max_regs()
+#ifndef QKN_LW_OVERLAP_REGS8
+#define QKN_LW_OVERLAP_REGS8 48
+#endif
+#ifndef QKN_LW_OVERLAP_REGS16
+#define QKN_LW_OVERLAP_REGS16 64
+#endif
+#ifndef QKN_LW_OVERLAP_REGS32
+#define QKN_LW_OVERLAP_REGS32 96
+#endif
+__host__ __device__ constexpr int layerwise_regs(int ept, bool overlap)
 {
-    constexpr int kEPT = VPT * Storage<TS>::kVec;
-    return kEPT <= 8 ? QKN_LW_REGS8 : (kEPT <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32);
+    return overlap ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
+                               : (ept <= 16 ? QKN_LW_OVERLAP_REGS16 : QKN_LW_OVERLAP_REGS32))
+                   : (ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32));
 }
 
-// Gamma in registers (at most 32 elements per thread).
-template <typename TS, int D, int VPT, bool kCluster, int kMode>
-__global__ void __maxnreg__((layerwise_max_regs<TS, VPT>()))
+// Gamma in registers (at most 32 elements per thread).  kOverlap: each
+// thread forms x * gamma while the token's partials are still being
+// combined (SwiftQK's overlap of the weight multiplication with the
+// exchange), so after the combine only the multiplication by the inverse RMS
+// remains, without a second pass over the staged token.
+template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap>
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kOverlap)))
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                      const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
                      float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
                      SumPlan plan_k, float *__restrict__ aux)
 {
-    layerwise_tokens<TS, D, VPT, true, kCluster, kMode>(qkv, row_stride, T, Hq, Hk, gamma_q,
-                                                        gamma_k, eps, inv_len_q, inv_len_k,
-                                                        plan_q, plan_k, aux);
+    layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kOverlap>(
+        qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
+        aux);
 }
 
 // Gamma read through L1 (tokens too wide for registers; one block per token,
@@ -695,9 +720,9 @@ qkn_layerwise_l1_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int
                         float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
                         SumPlan plan_k, float *__restrict__ aux)
 {
-    layerwise_tokens<TS, D, VPT, false, false, kMode>(qkv, row_stride, T, Hq, Hk, gamma_q,
-                                                      gamma_k, eps, inv_len_q, inv_len_k, plan_q,
-                                                      plan_k, aux);
+    layerwise_tokens<TS, D, VPT, false, false, kMode, false>(qkv, row_stride, T, Hq, Hk, gamma_q,
+                                                             gamma_k, eps, inv_len_q, inv_len_k,
+                                                             plan_q, plan_k, aux);
 }
 
 // ------------------------------------------------------------------- host --
@@ -885,7 +910,7 @@ constexpr bool layerwise_gamma_regs()
     return VPT * Storage<TS>::kVec <= 32;
 }
 
-template <typename TS, int D, int VPT, bool kCluster, int kMode>
+template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap = false>
 int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
                          const float *gq, const float *gk, float eps, int threads, int cluster,
                          float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
@@ -893,7 +918,7 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 {
     auto kern = [] {
         if constexpr (layerwise_gamma_regs<TS, VPT>())
-            return qkn_layerwise_kernel<TS, D, VPT, kCluster, kMode>;
+            return qkn_layerwise_kernel<TS, D, VPT, kCluster, kMode, kOverlap>;
         else
             return qkn_layerwise_l1_kernel<TS, D, VPT, kMode>;
     }();
@@ -953,15 +978,20 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 //    resident blocks, so more tokens are under way at once.
 // If no cluster size fits, one block per token with the fewest VPT within
 // 1024 threads, gamma read through L1 where it does not fit registers.
+// For fp32 and FP8 storage, a fused launch that is not short by the overlap
+// variant's own (larger) register count runs that variant: it saves the
+// second pass over the staged token, whose cost per element is highest
+// there (4 elements per 16-byte read for fp32, 16 conversions for FP8).
+// Measured on B200 it gained 1-7% on those shapes; for bf16 and fp16 and on
+// short inputs its extra registers cost more than the pass.
 constexpr int kLayerwiseMaxThreads = 576;
 constexpr int kLayerwiseShortTokens = 12;
 constexpr int kMaxCluster = 8;
 
-// Registers per thread of the gamma-in-registers kernel for `ept` elements
-// per thread (layerwise_max_regs at run time).
-int layerwise_regs(int ept)
+template <typename TS>
+constexpr bool layerwise_overlap_type()
 {
-    return ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32);
+    return Storage<TS>::kVec == 4 || Storage<TS>::kVec == 16;  // fp32, FP8
 }
 
 // Resident blocks per SM by the register file and the thread limit; the
@@ -1017,23 +1047,42 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
             }
         }
     }
-    if (chosen != 0 && 2 * chosen * kVec <= 32 && vpt_ok(2 * chosen)) {
+    bool overlap = false;
+    if (chosen != 0) {
         int dev = 0, rc;
         DeviceInfo info;
         if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
-        const int per_sm = layerwise_blocks_estimate(threads_for(cluster, chosen),
-                                                     layerwise_regs(chosen * kVec));
-        const int64_t pipelines = (int64_t)info.sms * per_sm / cluster;  // resident clusters
-        if (T < kLayerwiseShortTokens * pipelines) chosen *= 2;
+        // Resident clusters (token pipelines) with `regs` registers per thread.
+        auto pipelines = [&](int regs) {
+            const int per_sm = layerwise_blocks_estimate(threads_for(cluster, chosen), regs);
+            return (int64_t)info.sms * per_sm / cluster;
+        };
+        const int ept = chosen * kVec;
+        if (T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false))) {
+            if (2 * ept <= 32 && vpt_ok(2 * chosen)) chosen *= 2;
+        } else if (kMode == kFused && layerwise_overlap_type<TS>()) {
+            overlap = T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true));
+        }
     }
     for (int vpt = 1; vpt <= kNV && chosen == 0; vpt *= 2)
         if (vpt_ok(vpt) && threads_for(1, vpt) <= 1024) chosen = vpt;
     if (chosen == 0) return QKN_ERR_UNSUPPORTED;
     const int threads = (int)(((heads / cluster * (kNV / chosen)) + 31) / 32 * 32);
+    constexpr bool kMayOverlap = kMode == kFused && layerwise_overlap_type<TS>();
 #define QKN_LW_CASE(V)                                                                         \
     case V:                                                                                    \
         if constexpr (layerwise_vpt_ok<TS, D, V>()) {                                          \
             if constexpr (layerwise_gamma_regs<TS, V>()) {                                     \
+                if constexpr (kMayOverlap) {                                                   \
+                    if (overlap && cluster > 1)                                                \
+                        return launch_layerwise_vpt<TS, D, V, true, kMode, true>(              \
+                            qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, cluster,         \
+                            inv_len_q, inv_len_k, plan_q, plan_k, aux, stream);                \
+                    if (overlap)                                                               \
+                        return launch_layerwise_vpt<TS, D, V, false, kMode, true>(             \
+                            qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, 1, inv_len_q,    \
+                            inv_len_k, plan_q, plan_k, aux, stream);                           \
+                }                                                                              \
                 if (cluster > 1)                                                               \
                     return launch_layerwise_vpt<TS, D, V, true, kMode>(                        \
                         qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, cluster, inv_len_q,  \

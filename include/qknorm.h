@@ -18,9 +18,9 @@
  * Arithmetic: elements are widened to fp32, sums of squares accumulate in
  * fp32, the inverse RMS is 1/sqrt(S/L + eps) in fp32 (L = normalised length,
  * eps inside the square root; S/L is formed as S times 1/L rounded to fp32),
- * and each output x * rinv * gamma is rounded once to the storage type:
- * round to nearest even for bf16 and fp16, and for FP8 E4M3 round to nearest
- * even saturating to +-448.
+ * and each output, (x * rinv) * gamma per head and (x * gamma) * rinv
+ * layerwise, is rounded once to the storage type: round to nearest even for
+ * bf16 and fp16, and for FP8 E4M3 round to nearest even saturating to +-448.
  *
  * Common arguments
  *   qkv         device pointer to the fused buffer; 16-byte aligned.

@@ -63,6 +63,45 @@ def _tp_worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def _allgather_worker(rank, world, port, q):
+    """The All-Gather baseline's exchange: each rank holds its head shard of
+    every token's q and k; the gather must return the full vectors in head
+    order on every rank."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import attention_qk_norm_b200 as qkn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    T, Hq, Hk, D = 5, 8, 4, 16
+    x = torch.tensor(np.random.default_rng(1).standard_normal((T, (Hq + Hk) * D)))
+    xq, xk = x[:, :Hq * D], x[:, Hq * D:]
+    hq, hk = Hq // world, Hk // world
+    mine_q = xq[:, rank * hq * D:(rank + 1) * hq * D]
+    mine_k = xk[:, rank * hk * D:(rank + 1) * hk * D]
+    fq, fk, w, r = qkn.tp_allgather_full(mine_q, mine_k)
+    q.put((rank, w, r, bool(torch.equal(fq, xq)), bool(torch.equal(fk, xk))))
+    dist.destroy_process_group()
+
+
+def test_tensor_parallel_allgather_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_allgather_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == [(0, world, 0, True, True), (1, world, 1, True, True)]
+
+
 def test_tensor_parallel_allreduce_gloo():
     world = 2
     ctx = mp.get_context("spawn")

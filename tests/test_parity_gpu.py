@@ -346,6 +346,22 @@ def test_tensor_parallel_steps_emulated(Hq, Hk, D, dtype, n):
         assert np.array_equal(gu.stored_bits(x), out)
 
 
+@pytest.mark.parametrize("Hq,Hk,D,dtype", [(32, 8, 128, synth.BF16), (64, 8, 64, synth.FP32)])
+def test_tensor_parallel_allgather_baseline_one_rank(Hq, Hk, D, dtype):
+    """The All-Gather baseline with a single rank (no process group): the
+    gathered vectors are this rank's own, so the result is exactly the fused
+    kernel's, and V is untouched."""
+    c = synth.make_case(211, Hq, Hk, D, dtype=dtype, seed=95, layerwise=True, scale="lognormal")
+    x, gq, gk = gu.to_device(c)
+    qkn.qknorm_layerwise_tp_allgather(x, Hq, Hk, D, gq, gk, c.eps)
+    y, gq2, gk2 = gu.to_device(c)
+    qkn.qknorm_layerwise(y, Hq, Hk, D, gq2, gk2, c.eps)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.stored_bits(x), gu.stored_bits(y))
+    want = gu.oracle_out(c, "layerwise", c.qkv, c.T)
+    gu.check(gu.stored_bits(x), want, c.qkv, dtype, (Hq + Hk) * D, "all-gather baseline")
+
+
 def test_tensor_parallel_partials_leave_buffer_untouched():
     c = synth.make_case(77, 32, 8, 128, seed=90, layerwise=True)
     buf, _, _ = gu.to_device(c)
@@ -363,3 +379,46 @@ def test_no_in_kernel_wait_gave_up():
     its time limit (which would have left wrong results behind)."""
     torch.cuda.synchronize()
     assert qkn.wait_timeouts() == 0
+
+
+def test_calls_capture_into_a_cuda_graph():
+    """Decode-style use: a graph of per-head, layerwise and tensor-parallel
+    step calls, captured once and replayed on new inputs copied into the same
+    buffers, gives exactly the outputs of the same calls made eagerly (the
+    library neither allocates, synchronises nor reads device data on the host
+    inside a call)."""
+    Hq, Hk, D, T = 32, 8, 128, 3
+    cases = [synth.make_case(T, Hq, Hk, D, seed=s, layerwise=True) for s in (301, 302)]
+    x, gq, gk = gu.to_device(cases[0])      # per-head buffer
+    y, lq, lk = gu.to_device(cases[0])      # layerwise buffer (same data, other weights use)
+    z, _, _ = gu.to_device(cases[0])        # tensor-parallel steps buffer
+    gq_h, gk_h = gq[:D].contiguous(), gk[:D].contiguous()
+    part = torch.empty((T, 2), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm the launch-shape caches outside the capture
+        qkn.qknorm_per_head(x, Hq, Hk, D, gq_h, gk_h, 1e-6)
+        qkn.qknorm_layerwise(y, Hq, Hk, D, lq, lk, 1e-6, nshards=4)
+        qkn.qknorm_layerwise_partials(z, Hq, Hk, D, partials=part)
+        qkn.qknorm_layerwise_apply(z, Hq, Hk, D, lq, lk, part, Hq * D, Hk * D, 1e-6)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        qkn.qknorm_per_head(x, Hq, Hk, D, gq_h, gk_h, 1e-6)
+        qkn.qknorm_layerwise(y, Hq, Hk, D, lq, lk, 1e-6, nshards=4)
+        qkn.qknorm_layerwise_partials(z, Hq, Hk, D, partials=part)
+        qkn.qknorm_layerwise_apply(z, Hq, Hk, D, lq, lk, part, Hq * D, Hk * D, 1e-6)
+    for c in cases:
+        src, _, _ = gu.to_device(c)
+        for buf in (x, y, z):
+            buf.copy_(src)
+        g.replay()
+        torch.cuda.synchronize()
+        ex, _, _ = gu.to_device(c)
+        ey, _, _ = gu.to_device(c)
+        qkn.qknorm_per_head(ex, Hq, Hk, D, gq_h, gk_h, 1e-6)
+        qkn.qknorm_layerwise(ey, Hq, Hk, D, lq, lk, 1e-6, nshards=4)
+        torch.cuda.synchronize()
+        assert np.array_equal(gu.stored_bits(x), gu.stored_bits(ex))
+        assert np.array_equal(gu.stored_bits(y), gu.stored_bits(ey))
+        assert np.array_equal(gu.stored_bits(z), gu.stored_bits(ey))  # one rank: the fused result
