@@ -239,12 +239,18 @@ constexpr int per_head_min_blocks()
 // g + 2G, ... (G groups in the grid), U at a time.  The (token, head) pair of
 // each of its U rows is found once by division and then advanced by the fixed
 // step U*G with an add and one wrap, so the loop does no integer division.
-template <typename TS, int D, int U, bool kHasK>
+//
+// kSplit (used for FP8 with both kinds of heads): blocks [0, q_blocks) walk
+// the query rows only and the other blocks the key rows only, each with one
+// weight slice; holding both slices and selecting per element needs 80
+// registers for FP8's 16 elements per lane, one block per SM fewer.
+template <typename TS, int D, int U, bool kHasK, bool kSplit = false>
 __global__ void __launch_bounds__(kPerHeadThreads, (per_head_min_blocks<TS, D, kHasK>()))
 qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_t heads,
                     uint32_t Hq, const float *__restrict__ gamma_q,
-                    const float *__restrict__ gamma_k, float eps)
+                    const float *__restrict__ gamma_k, float eps, uint32_t q_blocks)
 {
+    static_assert(!(kSplit && kHasK), "a split block holds one weight");
     using S = Storage<TS>;
     using V = typename S::Vec;
     constexpr int kVec = S::kVec;
@@ -255,10 +261,23 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
     static_assert(32 % kLPR == 0 && kNV % kLPR == 0, "row must map onto a sub-warp");
 
     pdl_wait_then_release();
-    const uint64_t tid = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint64_t block = blockIdx.x, nblocks = gridDim.x;
+    if constexpr (kSplit) {
+        if (blockIdx.x >= q_blocks) {  // key rows: the columns after the Hq query heads
+            qkv += (int64_t)Hq * D;
+            gamma_q = gamma_k;
+            heads -= Hq;
+            block -= q_blocks;
+            nblocks -= q_blocks;
+        } else {
+            heads = Hq;
+            nblocks = q_blocks;
+        }
+    }
+    const uint64_t tid = block * blockDim.x + threadIdx.x;
     const uint32_t lane = (uint32_t)(tid % kLPR);
     const uint64_t group = tid / kLPR;
-    const uint64_t ngroups = ((uint64_t)gridDim.x * blockDim.x) / kLPR;
+    const uint64_t ngroups = (nblocks * blockDim.x) / kLPR;
 
     // This lane's columns are fixed: vectors lane, lane + LPR, ... of a row.
     float gq[kEPL], gk[kHasK ? kEPL : 1];
@@ -858,14 +877,14 @@ int resident_blocks(Kern kern, KernelCache &kc, int dev, const DeviceInfo &info,
     return QKN_OK;
 }
 
-template <typename TS, int D, bool kHasK>
+template <typename TS, int D, bool kHasK, bool kSplit = false>
 int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                       const float *gk, float eps, cudaStream_t stream)
 {
     constexpr int U = kPerHeadRowsInFlight;
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kLPR = kNV < 32 ? kNV : 32;
-    auto kern = qkn_per_head_kernel<TS, D, U, kHasK>;
+    auto kern = qkn_per_head_kernel<TS, D, U, kHasK, kSplit>;
     static KernelCache kc;
     int dev = 0, per_sm = 0, rc;
     DeviceInfo info;
@@ -873,23 +892,45 @@ int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, 
     if ((rc = resident_blocks(kern, kc, dev, info, kPerHeadThreads, 0, &per_sm)) != QKN_OK)
         return rc;
     if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
-    const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
     const uint64_t rows_per_block = (uint64_t)(kPerHeadThreads / kLPR) * U;
-    const uint64_t need = (rows + rows_per_block - 1) / rows_per_block;
-    const uint64_t cap = (uint64_t)info.sms * per_sm;
-    const unsigned grid = (unsigned)(need < cap ? need : cap);
-    return launch_pdl(kern, grid, kPerHeadThreads, 0, stream, 1u, static_cast<TS *>(qkv), row_stride, T,
-                      (uint32_t)(Hq + Hk), (uint32_t)Hq, gq, gk, eps);
+    uint64_t cap = (uint64_t)info.sms * per_sm;
+    const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
+    uint64_t grid = (rows + rows_per_block - 1) / rows_per_block, q_blocks = 0;
+    if constexpr (kSplit) {
+        // Blocks per segment: as many as its rows need; when both together
+        // exceed the resident capacity, the capacity split in proportion to
+        // the rows, at least one block each.
+        const uint64_t rq = (uint64_t)T * (uint64_t)Hq, rk = (uint64_t)T * (uint64_t)Hk;
+        uint64_t bq = (rq + rows_per_block - 1) / rows_per_block;
+        uint64_t bk = (rk + rows_per_block - 1) / rows_per_block;
+        if (cap < 2) cap = 2;
+        if (bq + bk > cap) {
+            bq = (cap * rq + (rq + rk) / 2) / (rq + rk);
+            if (bq < 1) bq = 1;
+            if (bq > cap - 1) bq = cap - 1;
+            bk = cap - bq;
+        }
+        grid = bq + bk;
+        q_blocks = bq;
+    } else if (grid > cap) {
+        grid = cap;
+    }
+    return launch_pdl(kern, (unsigned)grid, kPerHeadThreads, 0, stream, 1u,
+                      static_cast<TS *>(qkv), row_stride, T, (uint32_t)(Hq + Hk), (uint32_t)Hq, gq,
+                      gk, eps, (uint32_t)q_blocks);
 }
 
-// Only one weight is in use when a kind of head is absent: with no key heads
-// every row is a query row, and with no query heads every row is a key row.
 template <typename TS, int D>
 int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                     const float *gk, float eps, cudaStream_t stream)
 {
-    if (Hq > 0 && Hk > 0)
-        return launch_per_head_k<TS, D, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps, stream);
+    if (Hq > 0 && Hk > 0) {
+        if constexpr (Storage<TS>::kVec == 16)  // FP8
+            return launch_per_head_k<TS, D, false, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
+                                                          stream);
+        else
+            return launch_per_head_k<TS, D, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps, stream);
+    }
     const float *g = Hq > 0 ? gq : gk;
     return launch_per_head_k<TS, D, false>(qkv, T, Hq, Hk, row_stride, g, nullptr, eps, stream);
 }
