@@ -1019,12 +1019,13 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 //    resident blocks, so more tokens are under way at once.
 // If no cluster size fits, one block per token with the fewest VPT within
 // 1024 threads, gamma read through L1 where it does not fit registers.
-// For fp32 and FP8 storage, a fused launch that is not short by the overlap
-// variant's own (larger) register count runs that variant: it saves the
-// second pass over the staged token, whose cost per element is highest
-// there (4 elements per 16-byte read for fp32, 16 conversions for FP8).
-// Measured on B200 it gained 1-7% on those shapes; for bf16 and fp16 and on
-// short inputs its extra registers cost more than the pass.
+// For fp32 and FP8 storage, a fused launch that keeps its VPT and is not
+// short by the overlap variant's own (larger) register count runs that
+// variant: it saves the second pass over the staged token, whose cost per
+// element is highest there (4 elements per 16-byte read for fp32, 16
+// conversions for FP8).  Measured on B200 it gained 1-13% on those shapes;
+// for bf16 and fp16 and on short inputs its extra registers cost more than
+// the pass.
 constexpr int kLayerwiseMaxThreads = 576;
 constexpr int kLayerwiseShortTokens = 12;
 constexpr int kMaxCluster = 8;
@@ -1099,11 +1100,11 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
             return (int64_t)info.sms * per_sm / cluster;
         };
         const int ept = chosen * kVec;
-        if (T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false))) {
-            if (2 * ept <= 32 && vpt_ok(2 * chosen)) chosen *= 2;
-        } else if (kMode == kFused && layerwise_overlap_type<TS>()) {
+        const bool can_double = 2 * ept <= 32 && vpt_ok(2 * chosen);
+        if (can_double && T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false)))
+            chosen *= 2;
+        else if (kMode == kFused && layerwise_overlap_type<TS>())
             overlap = T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true));
-        }
     }
     for (int vpt = 1; vpt <= kNV && chosen == 0; vpt *= 2)
         if (vpt_ok(vpt) && threads_for(1, vpt) <= 1024) chosen = vpt;
