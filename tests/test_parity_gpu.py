@@ -243,6 +243,18 @@ def test_low_precision_layerwise(dtype, D, Hq, Hk):
     assert np.array_equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("dtype,T,Hq,Hk,D", [(synth.FP8, 8192, 32, 8, 128),
+                                              (synth.FP32, 4096, 64, 8, 64)])
+def test_layerwise_overlap_every_element(dtype, T, Hq, Hk, D):
+    """Inputs long enough for the launch rule to pick the overlap variant (x*gamma
+    formed before the combine): every element against the oracle, and the
+    same bits for every nshards."""
+    c = synth.make_case(T, Hq, Hk, D, dtype=dtype, seed=72 + D, layerwise=True, scale="stress",
+                        zero_frac=0.01, outlier_frac=0.01)
+    outs = [full_parity(c, "layerwise", n, what="overlap %s n=%d" % (dtype, n))[0] for n in (1, 8)]
+    assert np.array_equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("dtype", (synth.FP16, synth.FP8))
 def test_low_precision_full_size_sampled(dtype):
     d = synth.make_case_torch(16384, device="cuda", seed=70, **dict(synth.GQA, dtype=dtype))
