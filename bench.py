@@ -574,6 +574,8 @@ PROFILE_CASES = {
     "layerwise_wide": dict(kind="layerwise", T=8192, Hq=64, Hk=8, D=128, dtype="bf16", eps=1e-6,
                            nshards=8, scale="stress", zero_frac=0.01, outlier_frac=0.01,
                            seed=1004),
+    "layerwise_fp8": dict(kind="layerwise", T=32768, Hq=32, Hk=8, D=128, dtype="fp8_e4m3",
+                          eps=1e-6, nshards=8, seed=1006),
     # 128 heads of 256: too wide for one block, so 2-block clusters exchange
     # head partials through distributed shared memory.
     "layerwise_cluster": dict(kind="layerwise", T=4096, Hq=112, Hk=16, D=256, dtype="bf16",
