@@ -411,9 +411,17 @@ def cpu_baseline(w, budget_s=10.0):
         el = time.perf_counter() - t0
         if el >= budget_s or (passes >= 1 and el * (passes + 1) / passes > 3 * budget_s):
             break
+    # One host thread, on the first tokens only (bounded to a second or two).
+    n1 = min(c.T, 1024)
+    t1 = time.perf_counter()
+    oracle.per_head(c.qkv[:n1], c.dtype, n1, c.Hq, c.Hk, c.D, c.row_stride, c.gamma_q, c.gamma_k,
+                    c.eps, nthreads=1)
+    el1 = time.perf_counter() - t1
     return {"value": round(passes * c.T / el, 1), "unit": UNIT, "cores": threads,
             "kind": "oracle",
-            "sample": "%d full pass(es) of the %d-token workload (%.1f s)" % (passes, c.T, el)}
+            "sample": "%d full pass(es) of the %d-token workload (%.1f s)" % (passes, c.T, el),
+            "value_1_thread": round(n1 / el1, 1),
+            "sample_1_thread": "the first %d tokens on one host thread (%.2f s)" % (n1, el1)}
 
 
 # -------------------------------------------------------------- main arms --
