@@ -13,8 +13,10 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
-SOURCES = [os.path.join(PKG, "csrc", "qknorm.cu")]
-HEADERS = [os.path.join(INCLUDE, "qknorm.h")]
+CSRC = os.path.join(PKG, "csrc")
+SOURCES = [os.path.join(CSRC, "qknorm.cu")]
+HEADERS = [os.path.join(INCLUDE, "qknorm.h")] + sorted(
+    os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh"))
 LIB_PATH = os.path.join(PKG, "libqknorm.so")
 
 NVCC_FLAGS = [
@@ -29,6 +31,20 @@ def nvcc() -> str:
     if not os.path.exists(found):
         raise RuntimeError("nvcc not found; the CUDA toolkit is required to build libqknorm.so")
     return found
+
+
+def kernel_source_sha256() -> str:
+    """SHA-256 over the library's CUDA sources (file names and contents, in
+    name order); recorded ncu counters are valid only for the sources they
+    were taken from."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for p in sorted(SOURCES + HEADERS[1:]):
+        h.update(os.path.basename(p).encode() + b"\0")
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def is_stale() -> bool:

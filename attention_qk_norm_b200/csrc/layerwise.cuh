@@ -1,0 +1,404 @@
+// layerwise.cuh -- the layerwise QK-Norm kernel: the fixed reduction tree,
+// the cluster exchange of head partials on transaction barriers, and the
+// kernel entry points of its modes and variants.
+// Part of libqknorm.so; included by qknorm.cu, the library's one translation
+// unit.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "storage.cuh"
+
+namespace {
+
+// --------------------------------------------------------------- layerwise --
+constexpr int kLayerwiseStages = 2;
+
+// How warp_sumsq reduces the nh head partials of one vector (q or k).  The
+// host fills it once per launch, so the token loop divides nothing.
+//   used:      lanes that hold partials, min(p, 32) with p the largest power
+//              of two dividing nh (0 when nh == 0);
+//   per_lane:  heads each of those lanes sums, in order (nh / used);
+//   per_shard: lanes per emulated shard (used / nshards).
+struct SumPlan {
+    int used;
+    int per_lane;
+    int per_shard;
+};
+
+// Sum of squares of one vector from its head partials part[0..nh), computed
+// by one whole warp; every lane returns the same value.
+//
+// The reduction tree is fixed by nh alone: lane i sums heads
+// [i*per_lane, (i+1)*per_lane) in order, then xor butterflies join lanes at
+// distance 1, 2, 4, ...  With n shards (n a power of two dividing nh, so
+// n <= used), shard r holds exactly lanes [r*used/n, (r+1)*used/n): the
+// butterflies below distance used/n form each shard's partial S_r from that
+// shard's heads only, and the remaining ones are the scalar combine of
+// S_0..S_{n-1}.  So the result does not depend on n, bit for bit.
+__device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p, int lane)
+{
+    float v = 0.f;
+    if (lane < p.used)
+        for (int j = 0; j < p.per_lane; ++j) v += part[lane * p.per_lane + j];
+    for (int o = 1; o < p.per_shard; o <<= 1)  // rank-local partial S_r
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    for (int o = p.per_shard; o < p.used; o <<= 1)  // combine of the shard scalars
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return __shfl_sync(0xffffffffu, v, 0);
+}
+
+// ---- cluster exchange of head partials (transaction barriers) --
+// Each block of a cluster keeps two mbarriers, one per partials buffer.  The
+// owner of a head pushes that head's fp32 partial into the buffer of every
+// block of the cluster with st.async, which also counts its 4 bytes against
+// the receiving block's barrier; a block's barrier phase completes once all
+// (Hq + Hk) partials of the token have landed and its own thread 0 has armed
+// the phase.  No cluster-wide barrier and no memory fence is on the token path.
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(arrivals)
+                 : "memory");
+}
+// Make the initialised barriers visible to the other blocks of the cluster.
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// One arrival plus `bytes` expected transaction bytes for the current phase.
+__device__ __forceinline__ void mbar_arm(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// The shared::cluster address of `cta_addr` (a shared::cta address) in the
+// block of cluster rank `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t cta_addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(cta_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_async_f32(uint32_t dst, float v, uint32_t bar)
+{
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
+                     dst),
+                 "r"(__float_as_uint(v)), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits on a barrier give up after this long (they complete in microseconds
+// when the exchange works); each give-up is counted in g_wait_timeouts.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ unsigned int g_wait_timeouts;
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+// What a layerwise launch does with a token.
+//   kFused:    partial sums, scalar combine, inverse RMS and scaling, in place.
+//   kPartials: only this rank's two fp32 sums of squares (its q heads, its k
+//              heads), written to aux[2t], aux[2t+1]; the data is not written.
+//   kApply:    only the scaling, by 1/sqrt(aux[2t]/len_q + eps) for q and
+//              1/sqrt(aux[2t+1]/len_k + eps) for k, where aux holds the sums
+//              over all ranks and len_q, len_k the full vector lengths.
+// The mean S/L is formed as S * inv_len with inv_len = 1/L rounded to fp32
+// once per launch.
+enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
+
+// A token's heads are split over the CL blocks of a thread-block cluster
+// (CL = 1 for a plain launch): block c of a cluster owns heads
+// [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
+// thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
+// per head), and thread l == 0 is the head's owner.  Dynamic shared memory
+// per block: kLayerwiseStages stages of this block's part of a token
+// (hc*D*sizeof(TS) bytes), two buffers of `heads` fp32 head partials
+// (alternating per token), then the two exchange barriers (CL > 1).  With
+// CL = 1 the partials meet behind one block barrier per token; with CL > 1
+// each owner pushes its partial into every block of the cluster and each
+// block waits on its own barrier (see the exchange helpers above).
+template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode, bool kOverlap>
+__device__ __forceinline__ void
+layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                 const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
+                 float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
+                 float *__restrict__ aux)
+{
+    using S = Storage<TS>;
+    using V = typename S::Vec;
+    constexpr int kVB = (int)sizeof(V);  // bytes per vector
+    constexpr int kVec = S::kVec;
+    constexpr int kNV = D / kVec;     // vectors per head
+    constexpr int kLPH = kNV / VPT;   // threads per head
+    constexpr int kEPT = VPT * kVec;  // elements per thread
+    constexpr int NST = kLayerwiseStages;
+    constexpr bool kExchange = kCluster && kMode != kApply;
+    // Vector loops unroll fully when gamma sits in registers (indexed by v);
+    // with gamma in L1 the long loops unroll by 8.
+    constexpr int kUnroll = kGammaRegs || VPT < 8 ? VPT : 8;
+    static_assert(kNV % VPT == 0 && 32 % kLPH == 0, "head must map onto a sub-warp");
+
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int heads = Hq + Hk;
+    int cl = 1, crank = 0;
+    if constexpr (kCluster) {
+        cl = (int)cooperative_groups::this_cluster().num_blocks();
+        crank = (int)cooperative_groups::this_cluster().block_rank();
+    }
+    const int hc = heads / cl;           // heads of this block
+    const int h_lo = crank * hc;
+    const int span = hc * D * (int)sizeof(TS);
+    float *part = reinterpret_cast<float *>(smem + (size_t)NST * span);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(part + 2 * heads);
+    const uint32_t token_bytes = (uint32_t)heads * (uint32_t)sizeof(float);
+    const int hl = threadIdx.x / kLPH;   // head within this block
+    const int h = h_lo + hl;
+    const int l = threadIdx.x % kLPH;
+    const bool active = hl < hc;
+    const int lane = threadIdx.x % 32;
+    // Heads of this warp's threads; a warp computes only the inverse RMS of
+    // the vectors it holds (warp-uniform, so whole warps shuffle together).
+    const int warp_first_head = h_lo + (threadIdx.x & ~31) / kLPH;
+    const int warp_last_head = h_lo + (threadIdx.x | 31) / kLPH;
+    const bool need_q = warp_first_head < Hq;
+    const bool need_k = Hk > 0 && warp_last_head >= Hq;
+    const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
+
+    pdl_wait_then_release();
+    // This thread's head weights (the partials step has none).
+    const float *gb = gamma_q;
+    if (kMode != kPartials && active)
+        gb = h < Hq ? gamma_q + (int64_t)h * D : gamma_k + (int64_t)(h - Hq) * D;
+    float g[kGammaRegs ? kEPT : 1];
+#pragma unroll
+    for (int e = 0; e < (kGammaRegs ? kEPT : 1); ++e) g[e] = 0.f;
+    if (kGammaRegs && kMode != kPartials && active) {
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) {
+            float t4[kVec];
+            load_gamma<kVec>(gb + (l + v * kLPH) * kVec, t4);
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) g[v * kVec + e] = t4[e];
+        }
+    }
+    const int64_t col0 = (int64_t)h * D;          // in the token row
+    const int scol0 = (hl * D + l * kVec) * (int)sizeof(TS);  // in a stage
+    // Each thread copies, and later reads, only its own vectors of a stage.
+    auto fetch = [&](int64_t tok, int st) {
+        if (active && tok < T) {
+            const V *src = reinterpret_cast<const V *>(qkv + tok * row_stride + col0);
+            V *dst = reinterpret_cast<V *>(smem + (size_t)st * span + scol0);
+#pragma unroll kUnroll
+            for (int v = 0; v < VPT; ++v) cp_async<kVB>(dst + v * kLPH, src + l + v * kLPH);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
+    if constexpr (kExchange) {
+        if (threadIdx.x == 0) {
+            mbar_init(&bar[0], 1);
+            mbar_init(&bar[1], 1);
+            mbar_init_fence();
+            mbar_arm(&bar[0], token_bytes);
+            mbar_arm(&bar[1], token_bytes);
+        }
+        // Distributed shared memory may only be touched once every block of
+        // the cluster is running: meet once, barriers initialised and armed,
+        // before the first remote write.
+        cooperative_groups::this_cluster().sync();
+    }
+    int st = 0;
+    uint32_t it = 0;  // tokens this block has done; partials buffer it % 2
+    bool timed_out = false;
+    for (int64_t t = first; t < T; t += stride, ++it) {
+        // Refill the stage this thread finished with on the previous token.
+        fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
+        cp_async_wait<NST - 1>();
+        const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
+        float rq = 0.f, rk = 0.f;
+        float xg[kOverlap ? kEPT : 1];  // x * gamma, formed before the combine
+        if constexpr (kMode == kApply) {
+            // Sums over all ranks come in; no exchange inside the launch.
+            if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) * inv_len_q + eps);
+            if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) * inv_len_k + eps);
+        } else {
+            float s = 0.f;
+#pragma unroll kUnroll
+            for (int v = 0; v < VPT; ++v) {
+                float f[kVec];
+                S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
+#pragma unroll
+                for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
+                if constexpr (kOverlap) {
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) xg[v * kVec + e] = f[e] * g[v * kVec + e];
+                }
+            }
+            s = group_sum<kLPH>(s);
+            // Partials alternate between two buffers.  The next write into
+            // this token's buffer is for the token after next; every block
+            // sends it only after the token in between, which needs a partial
+            // from every warp of the cluster, and each warp sends that only
+            // after it has finished reading this buffer.  (Every warp holds an
+            // owner: its first thread.)
+            const uint32_t pb = it & 1u;
+            float *pp = part + pb * heads;
+            if constexpr (kExchange) {
+                if (active && l == 0) {
+                    const uint32_t dst = smem_u32(pp + h), b = smem_u32(&bar[pb]);
+                    for (int r = 0; r < cl; ++r)
+                        st_async_f32(cluster_addr(dst, (uint32_t)r), s,
+                                     cluster_addr(b, (uint32_t)r));
+                }
+                // Buffer pb serves every other token: phase it/2 of its barrier.
+                if (!timed_out && !mbar_wait_bounded(&bar[pb], (it >> 1) & 1u)) {
+                    timed_out = true;
+                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
+                }
+                // Arm the barrier's next phase (the token after next) before this
+                // thread sends its next partial, which any sender of that phase
+                // has to wait for.
+                if (threadIdx.x == 0 && !timed_out) mbar_arm(&bar[pb], token_bytes);
+            } else {
+                if (active && l == 0) pp[h] = s;
+                __syncthreads();
+            }
+            if constexpr (kMode == kPartials) {
+                // One warp of the cluster's first block writes this rank's sums.
+                if (threadIdx.x < 32 && crank == 0) {
+                    const float sq = warp_sumsq(pp, plan_q, lane);
+                    const float sk = warp_sumsq(pp + Hq, plan_k, lane);
+                    if (lane == 0) {
+                        aux[2 * t] = sq;
+                        aux[2 * t + 1] = sk;
+                    }
+                }
+            } else {
+                if (need_q) rq = rsqrtf(warp_sumsq(pp, plan_q, lane) * inv_len_q + eps);
+                if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, plan_k, lane) * inv_len_k + eps);
+            }
+        }
+        if (kMode != kPartials && active) {
+            const float rinv = h < Hq ? rq : rk;
+            V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
+#pragma unroll kUnroll
+            for (int v = 0; v < VPT; ++v) {
+                float o[kVec];
+                if constexpr (kOverlap) {
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) o[e] = xg[v * kVec + e] * rinv;
+                } else {
+                    float f[kVec], gv[kVec];
+                    S::unpack(sp[v * kLPH], f);
+                    if constexpr (kGammaRegs) {
+#pragma unroll
+                        for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
+                    } else {
+                        load_gamma<kVec>(gb + (l + v * kLPH) * kVec, gv);
+                    }
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) o[e] = f[e] * gv[e] * rinv;
+                }
+                store_stream(p + l + v * kLPH, S::pack(o));
+            }
+        }
+        st = (st + 1 == NST) ? 0 : st + 1;
+    }
+    cp_async_wait<0>();
+    // No block leaves while a partner could still write into it.
+    if constexpr (kExchange) cooperative_groups::this_cluster().sync();
+}
+
+// Registers per thread: 40, 48 or 56 when a thread keeps 8, 16 or 32
+// elements (and as many gamma values) per token.  The caps fit without
+// spilling and leave room for more resident blocks than the compiler's own
+// choice (up to 64); measured on B200 they are the fastest for every storage
+// type and head_dim.  The overlap variant also keeps the thread's x * gamma
+// products across the combine: 48, 64 or 96.
+#ifndef QKN_LW_REGS8
+#define QKN_LW_REGS8 40
+#endif
+#ifndef QKN_LW_REGS16
+#define QKN_LW_REGS16 48
+#endif
+#ifndef QKN_LW_REGS32
+#define QKN_LW_REGS32 56
+#endif
+#ifndef QKN_LW_OVERLAP_REGS8
+#define QKN_LW_OVERLAP_REGS8 48
+#endif
+#ifndef QKN_LW_OVERLAP_REGS16
+#define QKN_LW_OVERLAP_REGS16 64
+#endif
+#ifndef QKN_LW_OVERLAP_REGS32
+#define QKN_LW_OVERLAP_REGS32 96
+#endif
+__host__ __device__ constexpr int layerwise_regs(int ept, bool overlap)
+{
+    return overlap ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
+                               : (ept <= 16 ? QKN_LW_OVERLAP_REGS16 : QKN_LW_OVERLAP_REGS32))
+                   : (ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32));
+}
+
+// Gamma in registers (at most 32 elements per thread).  kOverlap: each
+// thread forms x * gamma while the token's partials are still being
+// combined (SwiftQK's overlap of the weight multiplication with the
+// exchange), so after the combine only the multiplication by the inverse RMS
+// remains, without a second pass over the staged token.
+template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap>
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kOverlap)))
+qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                     const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
+                     float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                     SumPlan plan_k, float *__restrict__ aux)
+{
+    layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kOverlap>(
+        qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
+        aux);
+}
+
+// Gamma read through L1 (tokens too wide for registers; one block per token,
+// up to 1024 threads).
+template <typename TS, int D, int VPT, int kMode>
+__global__ void __launch_bounds__(1024)
+qkn_layerwise_l1_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
+                        const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
+                        float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                        SumPlan plan_k, float *__restrict__ aux)
+{
+    layerwise_tokens<TS, D, VPT, false, false, kMode, false>(qkv, row_stride, T, Hq, Hk, gamma_q,
+                                                             gamma_k, eps, inv_len_q, inv_len_k,
+                                                             plan_q, plan_k, aux);
+}
+
+}  // namespace

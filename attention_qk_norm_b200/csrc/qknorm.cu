@@ -26,8 +26,13 @@
 // Both kernels are launched with programmatic dependent launch: they wait on
 // griddepcontrol.wait before their first global memory access, so a kernel
 // earlier in the stream always finishes first, and they allow the next
-// kernel to be scheduled as soon as all of their blocks are resident.  No
-// kernel here waits on another block, so none can hang.
+// kernel to be scheduled as soon as all of their blocks are resident.  The
+// only wait between blocks is inside a thread-block cluster of the layerwise
+// kernel, whose blocks the hardware schedules together; each such wait gives
+// up after a time limit, so no kernel here can hang.
+//
+// Files: storage.cuh (vectors and device helpers), per_head.cuh and
+// layerwise.cuh (the kernels), and this file (launch shapes and the C ABI).
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,729 +47,13 @@
 
 #include "qknorm.h"
 
+#include "layerwise.cuh"
+#include "per_head.cuh"
+#include "storage.cuh"
+
 namespace {
 
 constexpr int kMaxDevices = 64;
-
-// ---------------------------------------------------------------- vectors --
-template <typename TS>
-struct Storage;
-
-// Each storage type moves through memory in 16-byte vectors (type Vec) of
-// kVec elements: 8 for bf16 / fp16, 4 for fp32, 16 for FP8.  (8-byte vectors
-// for FP8, 8 elements like bf16, measured slower on B200.)
-template <>
-struct Storage<__nv_bfloat16> {
-    using Vec = uint4;
-    static constexpr int kVec = 8;  // elements per vector
-    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
-    {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
-    }
-    __device__ __forceinline__ static uint4 pack(const float (&f)[8])
-    {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t *>(&p);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
-};
-
-template <>
-struct Storage<float> {
-    using Vec = uint4;
-    static constexpr int kVec = 4;
-    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[4])
-    {
-        f[0] = __uint_as_float(v.x);
-        f[1] = __uint_as_float(v.y);
-        f[2] = __uint_as_float(v.z);
-        f[3] = __uint_as_float(v.w);
-    }
-    __device__ __forceinline__ static uint4 pack(const float (&f)[4])
-    {
-        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                          __float_as_uint(f[3]));
-    }
-};
-
-template <>
-struct Storage<__half> {
-    using Vec = uint4;
-    static constexpr int kVec = 8;
-    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
-    {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
-            f[2 * i] = p.x;
-            f[2 * i + 1] = p.y;
-        }
-    }
-    __device__ __forceinline__ static uint4 pack(const float (&f)[8])
-    {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            __half2 p = __floats2half2_rn(f[2 * i], f[2 * i + 1]);  // round to nearest even
-            w[i] = *reinterpret_cast<uint32_t *>(&p);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
-};
-
-// FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per 16-byte
-// vector.  Decoded exactly through fp16; encoded round-to-nearest-even,
-// saturating to +-448.  The lower byte of each pair is the earlier element.
-template <>
-struct Storage<__nv_fp8_e4m3> {
-    using Vec = uint4;
-    static constexpr int kVec = 16;
-    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[16])
-    {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
-                    (__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
-                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&r));
-                f[4 * i + 2 * j] = p.x;
-                f[4 * i + 2 * j + 1] = p.y;
-            }
-        }
-    }
-    __device__ __forceinline__ static uint4 pack(const float (&f)[16])
-    {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i], f[4 * i + 1]),
-                                                         __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i + 2], f[4 * i + 3]),
-                                                         __NV_SATFINITE, __NV_E4M3);
-            w[i] = lo | (hi << 16);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
-};
-
-// Streaming (evict-first) vector accesses: each element is touched once.
-__device__ __forceinline__ uint4 load_stream(const uint4 *p) { return __ldcs(p); }
-__device__ __forceinline__ void store_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
-
-template <typename V>
-__device__ __forceinline__ V zero_vec();
-template <>
-__device__ __forceinline__ uint4 zero_vec<uint4>() { return make_uint4(0u, 0u, 0u, 0u); }
-
-template <int N>
-__device__ __forceinline__ void load_gamma(const float *__restrict__ g, float (&out)[N])
-{
-    static_assert(N % 4 == 0, "gamma slices are whole float4s");
-#pragma unroll
-    for (int i = 0; i < N / 4; ++i) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(g) + i);
-        out[4 * i] = v.x;
-        out[4 * i + 1] = v.y;
-        out[4 * i + 2] = v.z;
-        out[4 * i + 3] = v.w;
-    }
-}
-
-// Sum over an aligned group of `kWidth` lanes (a power of two dividing 32).
-// With xor shuffles every lane ends with the same bits: each level adds the
-// same two operands, only in swapped order, and fp32 addition commutes.
-template <int kWidth>
-__device__ __forceinline__ float group_sum(float s)
-{
-#pragma unroll
-    for (int o = kWidth / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    return s;
-}
-
-// Programmatic dependent launch: wait for the grids this one depends on (all
-// their memory operations visible), then let dependents be scheduled.
-__device__ __forceinline__ void pdl_wait_then_release()
-{
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
-}
-
-// cp.async of one 16-byte vector into shared memory through L2 only (.cg),
-// in commit groups.  Each thread waits only for its own groups
-// (cp.async.wait_group), which the hardware completes; there is no spin loop.
-template <int kBytes>
-__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
-{
-    static_assert(kBytes == 16, "vectors are 16 bytes");
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// ---------------------------------------------------------------- per-head --
-constexpr int kPerHeadThreads = 256;
-constexpr int kPerHeadRowsInFlight = 2;
-// Resident 256-thread blocks per SM that the register budget must allow, by
-// elements a lane holds per row: six (40 registers) for the single-weight
-// loop with 8 elements, five (48) with both weights; four (64) and three (80)
-// for FP8's 16 elements; four for fp32 D=256 (two vectors per lane).  Each
-// fits without spilling.
-template <typename TS, int D, bool kHasK>
-constexpr int per_head_min_blocks()
-{
-    constexpr int kNV = D / Storage<TS>::kVec;
-    constexpr int kVPL = kNV > 32 ? kNV / 32 : 1;
-    constexpr int kEPL = kVPL * Storage<TS>::kVec;
-    return kVPL > 1 ? 4 : (kEPL > 8 ? (kHasK ? 3 : 4) : (kHasK ? 5 : 6));
-}
-
-// Rows are visited with a grid stride: thread group g takes rows g, g + G,
-// g + 2G, ... (G groups in the grid), U at a time.  The (token, head) pair of
-// each of its U rows is found once by division and then advanced by the fixed
-// step U*G with an add and one wrap, so the loop does no integer division.
-//
-// kSplit (used for FP8 with both kinds of heads): blocks [0, q_blocks) walk
-// the query rows only and the other blocks the key rows only, each with one
-// weight slice; holding both slices and selecting per element needs 80
-// registers for FP8's 16 elements per lane, one block per SM fewer.
-template <typename TS, int D, int U, bool kHasK, bool kSplit = false>
-__global__ void __launch_bounds__(kPerHeadThreads, (per_head_min_blocks<TS, D, kHasK>()))
-qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_t heads,
-                    uint32_t Hq, const float *__restrict__ gamma_q,
-                    const float *__restrict__ gamma_k, float eps, uint32_t q_blocks)
-{
-    static_assert(!(kSplit && kHasK), "a split block holds one weight");
-    using S = Storage<TS>;
-    using V = typename S::Vec;
-    constexpr int kVec = S::kVec;
-    constexpr int kNV = D / kVec;                  // vectors per row
-    constexpr int kLPR = kNV < 32 ? kNV : 32;      // lanes per row
-    constexpr int kVPL = kNV / kLPR;               // vectors per lane per row
-    constexpr int kEPL = kVPL * kVec;              // elements per lane per row
-    static_assert(32 % kLPR == 0 && kNV % kLPR == 0, "row must map onto a sub-warp");
-
-    pdl_wait_then_release();
-    uint64_t block = blockIdx.x, nblocks = gridDim.x;
-    if constexpr (kSplit) {
-        if (blockIdx.x >= q_blocks) {  // key rows: the columns after the Hq query heads
-            qkv += (int64_t)Hq * D;
-            gamma_q = gamma_k;
-            heads -= Hq;
-            block -= q_blocks;
-            nblocks -= q_blocks;
-        } else {
-            heads = Hq;
-            nblocks = q_blocks;
-        }
-    }
-    const uint64_t tid = block * blockDim.x + threadIdx.x;
-    const uint32_t lane = (uint32_t)(tid % kLPR);
-    const uint64_t group = tid / kLPR;
-    const uint64_t ngroups = (nblocks * blockDim.x) / kLPR;
-
-    // This lane's columns are fixed: vectors lane, lane + LPR, ... of a row.
-    float gq[kEPL], gk[kHasK ? kEPL : 1];
-#pragma unroll
-    for (int v = 0; v < kVPL; ++v) {
-        const int col = (lane + v * kLPR) * kVec;
-        float tq[kVec];
-        load_gamma<kVec>(gamma_q + col, tq);
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) gq[v * kVec + e] = tq[e];
-        if constexpr (kHasK) {
-            float tk[kVec];
-            load_gamma<kVec>(gamma_k + col, tk);
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) gk[v * kVec + e] = tk[e];
-        }
-    }
-
-    // The first rows and the step are below U * ngroups (at most a few
-    // hundred thousand), so 32-bit division can find their (token, head)
-    // pairs; it shortens the start of the single-weight kernel (measured
-    // 1.4% at the 48-head, 4096-token shape), while the two-weight variant
-    // measured faster with 64-bit division.
-    int64_t t[U];
-    uint32_t h[U];
-    const uint64_t step = ngroups * U;
-    int64_t dt;
-    uint32_t dh;
-    if constexpr (!kHasK) {
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const uint32_t r = (uint32_t)(k * ngroups + group);
-            const uint32_t q = r / heads;
-            t[k] = q;
-            h[k] = r - q * heads;
-        }
-        const uint32_t dt32 = (uint32_t)step / heads;
-        dt = dt32;
-        dh = (uint32_t)step - dt32 * heads;
-    } else {
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            const uint64_t r = (uint64_t)k * ngroups + group;
-            t[k] = (int64_t)(r / heads);
-            h[k] = (uint32_t)(r - (uint64_t)t[k] * heads);
-        }
-        dt = (int64_t)(step / heads);
-        dh = (uint32_t)(step - (uint64_t)dt * heads);
-    }
-    const uint64_t rows = (uint64_t)T * heads;
-    // The trip count is the same for every thread, so whole warps reach each
-    // shuffle together; rows past the end contribute zeros and store nothing.
-    for (uint64_t base = 0; base < rows; base += step) {
-        V x[U][kVPL];
-        V *ptr[U];
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            ptr[k] = reinterpret_cast<V *>(qkv + t[k] * row_stride + (int64_t)h[k] * D) + lane;
-#pragma unroll
-            for (int v = 0; v < kVPL; ++v)
-                x[k][v] = t[k] < T ? load_stream(ptr[k] + v * kLPR) : zero_vec<V>();
-        }
-#pragma unroll
-        for (int k = 0; k < U; ++k) {
-            float f[kVPL][kVec];
-            float s = 0.f;
-#pragma unroll
-            for (int v = 0; v < kVPL; ++v) {
-                S::unpack(x[k][v], f[v]);
-#pragma unroll
-                for (int e = 0; e < kVec; ++e) s = fmaf(f[v][e], f[v][e], s);
-            }
-            s = group_sum<kLPR>(s);
-            const float rinv = rsqrtf(s / (float)D + eps);
-            if (t[k] < T) {
-                const bool is_q = !kHasK || h[k] < Hq;
-#pragma unroll
-                for (int v = 0; v < kVPL; ++v) {
-                    float o[kVec];
-#pragma unroll
-                    for (int e = 0; e < kVec; ++e) {
-                        float g = gq[v * kVec + e];
-                        if constexpr (kHasK) g = is_q ? g : gk[v * kVec + e];
-                        o[e] = f[v][e] * rinv * g;
-                    }
-                    store_stream(ptr[k] + v * kLPR, S::pack(o));
-                }
-            }
-            h[k] += dh;
-            t[k] += dt;
-            if (h[k] >= heads) {
-                h[k] -= heads;
-                t[k] += 1;
-            }
-        }
-    }
-}
-
-// --------------------------------------------------------------- layerwise --
-constexpr int kLayerwiseStages = 2;
-
-// How warp_sumsq reduces the nh head partials of one vector (q or k).  The
-// host fills it once per launch, so the token loop divides nothing.
-//   used:      lanes that hold partials, min(p, 32) with p the largest power
-//              of two dividing nh (0 when nh == 0);
-//   per_lane:  heads each of those lanes sums, in order (nh / used);
-//   per_shard: lanes per emulated shard (used / nshards).
-struct SumPlan {
-    int used;
-    int per_lane;
-    int per_shard;
-};
-
-// Sum of squares of one vector from its head partials part[0..nh), computed
-// by one whole warp; every lane returns the same value.
-//
-// The reduction tree is fixed by nh alone: lane i sums heads
-// [i*per_lane, (i+1)*per_lane) in order, then xor butterflies join lanes at
-// distance 1, 2, 4, ...  With n shards (n a power of two dividing nh, so
-// n <= used), shard r holds exactly lanes [r*used/n, (r+1)*used/n): the
-// butterflies below distance used/n form each shard's partial S_r from that
-// shard's heads only, and the remaining ones are the scalar combine of
-// S_0..S_{n-1}.  So the result does not depend on n, bit for bit.
-__device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p, int lane)
-{
-    float v = 0.f;
-    if (lane < p.used)
-        for (int j = 0; j < p.per_lane; ++j) v += part[lane * p.per_lane + j];
-    for (int o = 1; o < p.per_shard; o <<= 1)  // rank-local partial S_r
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    for (int o = p.per_shard; o < p.used; o <<= 1)  // combine of the shard scalars
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    return __shfl_sync(0xffffffffu, v, 0);
-}
-
-// ---- cluster exchange of head partials (transaction barriers) --
-// Each block of a cluster keeps two mbarriers, one per partials buffer.  The
-// owner of a head pushes that head's fp32 partial into the buffer of every
-// block of the cluster with st.async, which also counts its 4 bytes against
-// the receiving block's barrier; a block's barrier phase completes once all
-// (Hq + Hk) partials of the token have landed and its own thread 0 has armed
-// the phase.  No cluster-wide barrier and no memory fence is on the token path.
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(arrivals)
-                 : "memory");
-}
-// Make the initialised barriers visible to the other blocks of the cluster.
-__device__ __forceinline__ void mbar_init_fence()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// One arrival plus `bytes` expected transaction bytes for the current phase.
-__device__ __forceinline__ void mbar_arm(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// The shared::cluster address of `cta_addr` (a shared::cta address) in the
-// block of cluster rank `rank`.
-__device__ __forceinline__ uint32_t cluster_addr(uint32_t cta_addr, uint32_t rank)
-{
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(cta_addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_async_f32(uint32_t dst, float v, uint32_t bar)
-{
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(
-                     dst),
-                 "r"(__float_as_uint(v)), "r"(bar)
-                 : "memory");
-}
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Waits on a barrier give up after this long (they complete in microseconds
-// when the exchange works); each give-up is counted in g_wait_timeouts.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ unsigned int g_wait_timeouts;
-
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > kWaitLimitNs) return false;
-    return true;
-}
-
-// What a layerwise launch does with a token.
-//   kFused:    partial sums, scalar combine, inverse RMS and scaling, in place.
-//   kPartials: only this rank's two fp32 sums of squares (its q heads, its k
-//              heads), written to aux[2t], aux[2t+1]; the data is not written.
-//   kApply:    only the scaling, by 1/sqrt(aux[2t]/len_q + eps) for q and
-//              1/sqrt(aux[2t+1]/len_k + eps) for k, where aux holds the sums
-//              over all ranks and len_q, len_k the full vector lengths.
-// The mean S/L is formed as S * inv_len with inv_len = 1/L rounded to fp32
-// once per launch.
-enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
-
-// A token's heads are split over the CL blocks of a thread-block cluster
-// (CL = 1 for a plain launch): block c of a cluster owns heads
-// [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
-// thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
-// per head), and thread l == 0 is the head's owner.  Dynamic shared memory
-// per block: kLayerwiseStages stages of this block's part of a token
-// (hc*D*sizeof(TS) bytes), two buffers of `heads` fp32 head partials
-// (alternating per token), then the two exchange barriers (CL > 1).  With
-// CL = 1 the partials meet behind one block barrier per token; with CL > 1
-// each owner pushes its partial into every block of the cluster and each
-// block waits on its own barrier (see the exchange helpers above).
-template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode, bool kOverlap>
-__device__ __forceinline__ void
-layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
-                 const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
-                 float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
-                 float *__restrict__ aux)
-{
-    using S = Storage<TS>;
-    using V = typename S::Vec;
-    constexpr int kVB = (int)sizeof(V);  // bytes per vector
-    constexpr int kVec = S::kVec;
-    constexpr int kNV = D / kVec;     // vectors per head
-    constexpr int kLPH = kNV / VPT;   // threads per head
-    constexpr int kEPT = VPT * kVec;  // elements per thread
-    constexpr int NST = kLayerwiseStages;
-    constexpr bool kExchange = kCluster && kMode != kApply;
-    // Vector loops unroll fully when gamma sits in registers (indexed by v);
-    // with gamma in L1 the long loops unroll by 8.
-    constexpr int kUnroll = kGammaRegs || VPT < 8 ? VPT : 8;
-    static_assert(kNV % VPT == 0 && 32 % kLPH == 0, "head must map onto a sub-warp");
-
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int heads = Hq + Hk;
-    int cl = 1, crank = 0;
-    if constexpr (kCluster) {
-        cl = (int)cooperative_groups::this_cluster().num_blocks();
-        crank = (int)cooperative_groups::this_cluster().block_rank();
-    }
-    const int hc = heads / cl;           // heads of this block
-    const int h_lo = crank * hc;
-    const int span = hc * D * (int)sizeof(TS);
-    float *part = reinterpret_cast<float *>(smem + (size_t)NST * span);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(part + 2 * heads);
-    const uint32_t token_bytes = (uint32_t)heads * (uint32_t)sizeof(float);
-    const int hl = threadIdx.x / kLPH;   // head within this block
-    const int h = h_lo + hl;
-    const int l = threadIdx.x % kLPH;
-    const bool active = hl < hc;
-    const int lane = threadIdx.x % 32;
-    // Heads of this warp's threads; a warp computes only the inverse RMS of
-    // the vectors it holds (warp-uniform, so whole warps shuffle together).
-    const int warp_first_head = h_lo + (threadIdx.x & ~31) / kLPH;
-    const int warp_last_head = h_lo + (threadIdx.x | 31) / kLPH;
-    const bool need_q = warp_first_head < Hq;
-    const bool need_k = Hk > 0 && warp_last_head >= Hq;
-    const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
-
-    pdl_wait_then_release();
-    // This thread's head weights (the partials step has none).
-    const float *gb = gamma_q;
-    if (kMode != kPartials && active)
-        gb = h < Hq ? gamma_q + (int64_t)h * D : gamma_k + (int64_t)(h - Hq) * D;
-    float g[kGammaRegs ? kEPT : 1];
-#pragma unroll
-    for (int e = 0; e < (kGammaRegs ? kEPT : 1); ++e) g[e] = 0.f;
-    if (kGammaRegs && kMode != kPartials && active) {
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) {
-            float t4[kVec];
-            load_gamma<kVec>(gb + (l + v * kLPH) * kVec, t4);
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) g[v * kVec + e] = t4[e];
-        }
-    }
-    const int64_t col0 = (int64_t)h * D;          // in the token row
-    const int scol0 = (hl * D + l * kVec) * (int)sizeof(TS);  // in a stage
-    // Each thread copies, and later reads, only its own vectors of a stage.
-    auto fetch = [&](int64_t tok, int st) {
-        if (active && tok < T) {
-            const V *src = reinterpret_cast<const V *>(qkv + tok * row_stride + col0);
-            V *dst = reinterpret_cast<V *>(smem + (size_t)st * span + scol0);
-#pragma unroll kUnroll
-            for (int v = 0; v < VPT; ++v) cp_async<kVB>(dst + v * kLPH, src + l + v * kLPH);
-        }
-        cp_async_commit();
-    };
-#pragma unroll
-    for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
-    if constexpr (kExchange) {
-        if (threadIdx.x == 0) {
-            mbar_init(&bar[0], 1);
-            mbar_init(&bar[1], 1);
-            mbar_init_fence();
-            mbar_arm(&bar[0], token_bytes);
-            mbar_arm(&bar[1], token_bytes);
-        }
-        // Distributed shared memory may only be touched once every block of
-        // the cluster is running: meet once, barriers initialised and armed,
-        // before the first remote write.
-        cooperative_groups::this_cluster().sync();
-    }
-    int st = 0;
-    uint32_t it = 0;  // tokens this block has done; partials buffer it % 2
-    bool timed_out = false;
-    for (int64_t t = first; t < T; t += stride, ++it) {
-        // Refill the stage this thread finished with on the previous token.
-        fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
-        cp_async_wait<NST - 1>();
-        const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
-        float rq = 0.f, rk = 0.f;
-        float xg[kOverlap ? kEPT : 1];  // x * gamma, formed before the combine
-        if constexpr (kMode == kApply) {
-            // Sums over all ranks come in; no exchange inside the launch.
-            if (Hq > 0) rq = rsqrtf(__ldg(aux + 2 * t) * inv_len_q + eps);
-            if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) * inv_len_k + eps);
-        } else {
-            float s = 0.f;
-#pragma unroll kUnroll
-            for (int v = 0; v < VPT; ++v) {
-                float f[kVec];
-                S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
-#pragma unroll
-                for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
-                if constexpr (kOverlap) {
-#pragma unroll
-                    for (int e = 0; e < kVec; ++e) xg[v * kVec + e] = f[e] * g[v * kVec + e];
-                }
-            }
-            s = group_sum<kLPH>(s);
-            // Partials alternate between two buffers.  The next write into
-            // this token's buffer is for the token after next; every block
-            // sends it only after the token in between, which needs a partial
-            // from every warp of the cluster, and each warp sends that only
-            // after it has finished reading this buffer.  (Every warp holds an
-            // owner: its first thread.)
-            const uint32_t pb = it & 1u;
-            float *pp = part + pb * heads;
-            if constexpr (kExchange) {
-                if (active && l == 0) {
-                    const uint32_t dst = smem_u32(pp + h), b = smem_u32(&bar[pb]);
-                    for (int r = 0; r < cl; ++r)
-                        st_async_f32(cluster_addr(dst, (uint32_t)r), s,
-                                     cluster_addr(b, (uint32_t)r));
-                }
-                // Buffer pb serves every other token: phase it/2 of its barrier.
-                if (!timed_out && !mbar_wait_bounded(&bar[pb], (it >> 1) & 1u)) {
-                    timed_out = true;
-                    if (lane == 0) atomicAdd(&g_wait_timeouts, 1u);
-                }
-                // Arm the barrier's next phase (the token after next) before this
-                // thread sends its next partial, which any sender of that phase
-                // has to wait for.
-                if (threadIdx.x == 0 && !timed_out) mbar_arm(&bar[pb], token_bytes);
-            } else {
-                if (active && l == 0) pp[h] = s;
-                __syncthreads();
-            }
-            if constexpr (kMode == kPartials) {
-                // One warp of the cluster's first block writes this rank's sums.
-                if (threadIdx.x < 32 && crank == 0) {
-                    const float sq = warp_sumsq(pp, plan_q, lane);
-                    const float sk = warp_sumsq(pp + Hq, plan_k, lane);
-                    if (lane == 0) {
-                        aux[2 * t] = sq;
-                        aux[2 * t + 1] = sk;
-                    }
-                }
-            } else {
-                if (need_q) rq = rsqrtf(warp_sumsq(pp, plan_q, lane) * inv_len_q + eps);
-                if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, plan_k, lane) * inv_len_k + eps);
-            }
-        }
-        if (kMode != kPartials && active) {
-            const float rinv = h < Hq ? rq : rk;
-            V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
-#pragma unroll kUnroll
-            for (int v = 0; v < VPT; ++v) {
-                float o[kVec];
-                if constexpr (kOverlap) {
-#pragma unroll
-                    for (int e = 0; e < kVec; ++e) o[e] = xg[v * kVec + e] * rinv;
-                } else {
-                    float f[kVec], gv[kVec];
-                    S::unpack(sp[v * kLPH], f);
-                    if constexpr (kGammaRegs) {
-#pragma unroll
-                        for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
-                    } else {
-                        load_gamma<kVec>(gb + (l + v * kLPH) * kVec, gv);
-                    }
-#pragma unroll
-                    for (int e = 0; e < kVec; ++e) o[e] = f[e] * gv[e] * rinv;
-                }
-                store_stream(p + l + v * kLPH, S::pack(o));
-            }
-        }
-        st = (st + 1 == NST) ? 0 : st + 1;
-    }
-    cp_async_wait<0>();
-    // No block leaves while a partner could still write into it.
-    if constexpr (kExchange) cooperative_groups::this_cluster().sync();
-}
-
-// Registers per thread: 40, 48 or 56 when a thread keeps 8, 16 or 32
-// elements (and as many gamma values) per token.  The caps fit without
-// spilling and leave room for more resident blocks than the compiler's own
-// choice (up to 64); measured on B200 they are the fastest for every storage
-// type and head_dim.  The overlap variant also keeps the thread's x * gamma
-// products across the combine: 48, 64 or 96.
-#ifndef QKN_LW_REGS8
-#define QKN_LW_REGS8 40
-#endif
-#ifndef QKN_LW_REGS16
-#define QKN_LW_REGS16 48
-#endif
-#ifndef QKN_LW_REGS32
-#define QKN_LW_REGS32 56
-#endif
-#ifndef QKN_LW_OVERLAP_REGS8
-#define QKN_LW_OVERLAP_REGS8 48
-#endif
-#ifndef QKN_LW_OVERLAP_REGS16
-#define QKN_LW_OVERLAP_REGS16 64
-#endif
-#ifndef QKN_LW_OVERLAP_REGS32
-#define QKN_LW_OVERLAP_REGS32 96
-#endif
-__host__ __device__ constexpr int layerwise_regs(int ept, bool overlap)
-{
-    return overlap ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
-                               : (ept <= 16 ? QKN_LW_OVERLAP_REGS16 : QKN_LW_OVERLAP_REGS32))
-                   : (ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32));
-}
-
-// Gamma in registers (at most 32 elements per thread).  kOverlap: each
-// thread forms x * gamma while the token's partials are still being
-// combined (SwiftQK's overlap of the weight multiplication with the
-// exchange), so after the combine only the multiplication by the inverse RMS
-// remains, without a second pass over the staged token.
-template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap>
-__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kOverlap)))
-qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
-                     const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
-                     float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
-                     SumPlan plan_k, float *__restrict__ aux)
-{
-    layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kOverlap>(
-        qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
-        aux);
-}
-
-// Gamma read through L1 (tokens too wide for registers; one block per token,
-// up to 1024 threads).
-template <typename TS, int D, int VPT, int kMode>
-__global__ void __launch_bounds__(1024)
-qkn_layerwise_l1_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
-                        const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
-                        float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
-                        SumPlan plan_k, float *__restrict__ aux)
-{
-    layerwise_tokens<TS, D, VPT, false, false, kMode, false>(qkv, row_stride, T, Hq, Hk, gamma_q,
-                                                             gamma_k, eps, inv_len_q, inv_len_k,
-                                                             plan_q, plan_k, aux);
-}
 
 // ------------------------------------------------------------------- host --
 thread_local int g_last_cuda_error = 0;

@@ -1,0 +1,186 @@
+// storage.cuh -- 16-byte vectors of each storage type, streaming accesses,
+// sub-warp sums, programmatic dependent launch and cp.async helpers.
+// Part of libqknorm.so; included by qknorm.cu, the library's one translation
+// unit.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace {
+
+// ---------------------------------------------------------------- vectors --
+template <typename TS>
+struct Storage;
+
+// Each storage type moves through memory in 16-byte vectors (type Vec) of
+// kVec elements: 8 for bf16 / fp16, 4 for fp32, 16 for FP8.  (8-byte vectors
+// for FP8, 8 elements like bf16, measured slower on B200.)
+template <>
+struct Storage<__nv_bfloat16> {
+    using Vec = uint4;
+    static constexpr int kVec = 8;  // elements per vector
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[8])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t *>(&p);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <>
+struct Storage<float> {
+    using Vec = uint4;
+    static constexpr int kVec = 4;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[4])
+    {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[4])
+    {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+
+template <>
+struct Storage<__half> {
+    using Vec = uint4;
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[8])
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            f[2 * i] = p.x;
+            f[2 * i + 1] = p.y;
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[8])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2 p = __floats2half2_rn(f[2 * i], f[2 * i + 1]);  // round to nearest even
+            w[i] = *reinterpret_cast<uint32_t *>(&p);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+// FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per 16-byte
+// vector.  Decoded exactly through fp16; encoded round-to-nearest-even,
+// saturating to +-448.  The lower byte of each pair is the earlier element.
+template <>
+struct Storage<__nv_fp8_e4m3> {
+    using Vec = uint4;
+    static constexpr int kVec = 16;
+    __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[16])
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
+                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&r));
+                f[4 * i + 2 * j] = p.x;
+                f[4 * i + 2 * j + 1] = p.y;
+            }
+        }
+    }
+    __device__ __forceinline__ static uint4 pack(const float (&f)[16])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i], f[4 * i + 1]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i + 2], f[4 * i + 3]),
+                                                         __NV_SATFINITE, __NV_E4M3);
+            w[i] = lo | (hi << 16);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+// Streaming (evict-first) vector accesses: each element is touched once.
+__device__ __forceinline__ uint4 load_stream(const uint4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void store_stream(uint4 *p, const uint4 &v) { __stcs(p, v); }
+
+template <typename V>
+__device__ __forceinline__ V zero_vec();
+template <>
+__device__ __forceinline__ uint4 zero_vec<uint4>() { return make_uint4(0u, 0u, 0u, 0u); }
+
+template <int N>
+__device__ __forceinline__ void load_gamma(const float *__restrict__ g, float (&out)[N])
+{
+    static_assert(N % 4 == 0, "gamma slices are whole float4s");
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(g) + i);
+        out[4 * i] = v.x;
+        out[4 * i + 1] = v.y;
+        out[4 * i + 2] = v.z;
+        out[4 * i + 3] = v.w;
+    }
+}
+
+// Sum over an aligned group of `kWidth` lanes (a power of two dividing 32).
+// With xor shuffles every lane ends with the same bits: each level adds the
+// same two operands, only in swapped order, and fp32 addition commutes.
+template <int kWidth>
+__device__ __forceinline__ float group_sum(float s)
+{
+#pragma unroll
+    for (int o = kWidth / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// Programmatic dependent launch: wait for the grids this one depends on (all
+// their memory operations visible), then let dependents be scheduled.
+__device__ __forceinline__ void pdl_wait_then_release()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
+// cp.async of one 16-byte vector into shared memory through L2 only (.cg),
+// in commit groups.  Each thread waits only for its own groups
+// (cp.async.wait_group), which the hardware completes; there is no spin loop.
+template <int kBytes>
+__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
+{
+    static_assert(kBytes == 16, "vectors are 16 bytes");
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+}  // namespace

@@ -28,7 +28,6 @@ data; NCCL carries only the barrier and the max of the timings).
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import math
 import os
@@ -85,16 +84,15 @@ def peaks():
 
 
 def traffic_record():
-    """Committed ncu DRAM bytes per launch, valid only for the kernel source
-    they were taken from (hash of csrc/qknorm.cu)."""
+    """Committed ncu DRAM bytes per launch, valid only for the kernel sources
+    they were taken from (buildlib.kernel_source_sha256)."""
+    from attention_qk_norm_b200 import buildlib
+
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "attention_qk_norm_b200", "csrc", "qknorm.cu")
     try:
         with open(path) as f:
             rec = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        return rec if rec.get("source_sha256") == sha else None
+        return rec if rec.get("source_sha256") == buildlib.kernel_source_sha256() else None
     except Exception:
         return None
 
