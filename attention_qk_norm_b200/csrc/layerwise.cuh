@@ -135,6 +135,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 // once per launch.
 enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 
+// How a launch moves each token through its block.
+//   kSchedRing:    a two-stage cp.async ring in shared memory (the next token
+//                  is fetched while this one is processed), then a second pass
+//                  over the staged token to scale it.
+//   kSchedOverlap: the ring, with x * gamma formed in the first pass, while
+//                  the token's partials are still being combined (SwiftQK's
+//                  overlap), and kept in registers: no second pass.
+//   kSchedDirect:  for launches where every cluster has about one token, so
+//                  there is nothing to prefetch: each thread loads its vectors
+//                  straight into registers and scales them there; nothing is
+//                  staged.
+enum LayerwiseSchedule { kSchedRing = 0, kSchedOverlap = 1, kSchedDirect = 2 };
+
 // A token's heads are split over the CL blocks of a thread-block cluster
 // (CL = 1 for a plain launch): block c of a cluster owns heads
 // [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
@@ -146,7 +159,7 @@ enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 // CL = 1 the partials meet behind one block barrier per token; with CL > 1
 // each owner pushes its partial into every block of the cluster and each
 // block waits on its own barrier (see the exchange helpers above).
-template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode, bool kOverlap>
+template <typename TS, int D, int VPT, bool kGammaRegs, bool kCluster, int kMode, int kSched>
 __device__ __forceinline__ void
 layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                  const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
@@ -160,7 +173,9 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     constexpr int kNV = D / kVec;     // vectors per head
     constexpr int kLPH = kNV / VPT;   // threads per head
     constexpr int kEPT = VPT * kVec;  // elements per thread
-    constexpr int NST = kLayerwiseStages;
+    constexpr bool kOverlap = kSched == kSchedOverlap;
+    constexpr bool kDirect = kSched == kSchedDirect;
+    constexpr int NST = kDirect ? 0 : kLayerwiseStages;  // stages of the ring
     constexpr bool kExchange = kCluster && kMode != kApply;
     // Vector loops unroll fully when gamma sits in registers (indexed by v);
     // with gamma in L1 the long loops unroll by 8.
@@ -222,8 +237,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
         }
         cp_async_commit();
     };
+    if constexpr (!kDirect) {
 #pragma unroll
-    for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
+        for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
+    }
     if constexpr (kExchange) {
         if (threadIdx.x == 0) {
             mbar_init(&bar[0], 1);
@@ -241,10 +258,19 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     uint32_t it = 0;  // tokens this block has done; partials buffer it % 2
     bool timed_out = false;
     for (int64_t t = first; t < T; t += stride, ++it) {
-        // Refill the stage this thread finished with on the previous token.
-        fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
-        cp_async_wait<NST - 1>();
-        const V *sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
+        const V *sp = nullptr;  // this thread's vectors of the token, staged (ring)
+        V xr[kDirect ? VPT : 1];  // or in registers (direct)
+        if constexpr (kDirect) {
+            const V *src = reinterpret_cast<const V *>(qkv + t * row_stride + col0);
+#pragma unroll
+            for (int v = 0; v < VPT; ++v)
+                xr[v] = active ? load_stream(src + l + v * kLPH) : zero_vec<V>();
+        } else {
+            // Refill the stage this thread finished with on the previous token.
+            fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
+            cp_async_wait<NST - 1>();
+            sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
+        }
         float rq = 0.f, rk = 0.f;
         float xg[kOverlap ? kEPT : 1];  // x * gamma, formed before the combine
         if constexpr (kMode == kApply) {
@@ -256,7 +282,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec];
-                S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
+                if constexpr (kDirect)
+                    S::unpack(xr[v], f);
+                else
+                    S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
 #pragma unroll
                 for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
                 if constexpr (kOverlap) {
@@ -319,7 +348,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                     for (int e = 0; e < kVec; ++e) o[e] = xg[v * kVec + e] * rinv;
                 } else {
                     float f[kVec], gv[kVec];
-                    S::unpack(sp[v * kLPH], f);
+                    if constexpr (kDirect)
+                        S::unpack(xr[v], f);
+                    else
+                        S::unpack(sp[v * kLPH], f);
                     if constexpr (kGammaRegs) {
 #pragma unroll
                         for (int e = 0; e < kVec; ++e) gv[e] = g[v * kVec + e];
@@ -332,7 +364,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 store_stream(p + l + v * kLPH, S::pack(o));
             }
         }
-        st = (st + 1 == NST) ? 0 : st + 1;
+        if constexpr (!kDirect) st = (st + 1 == NST) ? 0 : st + 1;
     }
     cp_async_wait<0>();
     // No block leaves while a partner could still write into it.
@@ -343,8 +375,8 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 // elements (and as many gamma values) per token.  The caps fit without
 // spilling and leave room for more resident blocks than the compiler's own
 // choice (up to 64); measured on B200 they are the fastest for every storage
-// type and head_dim.  The overlap variant also keeps the thread's x * gamma
-// products across the combine: 48, 64 or 96.
+// type and head_dim.  The overlap and direct schedules also keep the thread's
+// x * gamma products, or its raw vectors, in registers: 48, 64 or 96.
 #ifndef QKN_LW_REGS8
 #define QKN_LW_REGS8 40
 #endif
@@ -363,26 +395,26 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #ifndef QKN_LW_OVERLAP_REGS32
 #define QKN_LW_OVERLAP_REGS32 96
 #endif
-__host__ __device__ constexpr int layerwise_regs(int ept, bool overlap)
+__host__ __device__ constexpr int layerwise_regs(int ept, bool wide)
 {
-    return overlap ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
+    return wide ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
                                : (ept <= 16 ? QKN_LW_OVERLAP_REGS16 : QKN_LW_OVERLAP_REGS32))
                    : (ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32));
 }
 
-// Gamma in registers (at most 32 elements per thread).  kOverlap: each
-// thread forms x * gamma while the token's partials are still being
-// combined (SwiftQK's overlap of the weight multiplication with the
-// exchange), so after the combine only the multiplication by the inverse RMS
-// remains, without a second pass over the staged token.
-template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap>
-__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kOverlap)))
+// Gamma in registers (at most 32 elements per thread), with schedule kSched
+// (LayerwiseSchedule).  With kSchedOverlap each thread forms x * gamma while
+// the token's partials are still being combined (SwiftQK's overlap of the
+// weight multiplication with the exchange), so after the combine only the
+// multiplication by the inverse RMS remains.
+template <typename TS, int D, int VPT, bool kCluster, int kMode, int kSched>
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kSched != kSchedRing)))
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                      const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
                      float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
                      SumPlan plan_k, float *__restrict__ aux)
 {
-    layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kOverlap>(
+    layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kSched>(
         qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
         aux);
 }
@@ -396,9 +428,9 @@ qkn_layerwise_l1_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int
                         float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
                         SumPlan plan_k, float *__restrict__ aux)
 {
-    layerwise_tokens<TS, D, VPT, false, false, kMode, false>(qkv, row_stride, T, Hq, Hk, gamma_q,
-                                                             gamma_k, eps, inv_len_q, inv_len_k,
-                                                             plan_q, plan_k, aux);
+    layerwise_tokens<TS, D, VPT, false, false, kMode, kSchedRing>(
+        qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
+        aux);
 }
 
 }  // namespace

@@ -262,7 +262,7 @@ constexpr bool layerwise_gamma_regs()
     return VPT * Storage<TS>::kVec <= 32;
 }
 
-template <typename TS, int D, int VPT, bool kCluster, int kMode, bool kOverlap = false>
+template <typename TS, int D, int VPT, bool kCluster, int kMode, int kSched = kSchedRing>
 int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
                          const float *gq, const float *gk, float eps, int threads, int cluster,
                          float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
@@ -270,15 +270,15 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 {
     auto kern = [] {
         if constexpr (layerwise_gamma_regs<TS, VPT>())
-            return qkn_layerwise_kernel<TS, D, VPT, kCluster, kMode, kOverlap>;
+            return qkn_layerwise_kernel<TS, D, VPT, kCluster, kMode, kSched>;
         else
             return qkn_layerwise_l1_kernel<TS, D, VPT, kMode>;
     }();
     static KernelCache kc;
     const int heads = Hq + Hk;
     const size_t span = (size_t)(heads / cluster) * D * sizeof(TS);
-    const size_t smem =
-        kLayerwiseStages * span + (size_t)2 * heads * sizeof(float) + 2 * sizeof(uint64_t);
+    const size_t stages = kSched == kSchedDirect ? 0 : kLayerwiseStages;
+    const size_t smem = stages * span + (size_t)2 * heads * sizeof(float) + 2 * sizeof(uint64_t);
     int dev = 0, rc;
     DeviceInfo info;
     if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
@@ -318,6 +318,44 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
                       eps, inv_len_q, inv_len_k, plan_q, plan_k, aux);
 }
 
+// Storage types whose large fused launches use the overlap schedule.
+template <typename TS>
+constexpr bool layerwise_overlap_type()
+{
+    return Storage<TS>::kVec == 4 || Storage<TS>::kVec == 16;  // fp32, FP8
+}
+
+// The kernel instance for one vectors-per-thread count: the schedule (only
+// fused launches use the direct and overlap ones, and the overlap only for
+// fp32 and FP8) and whether the launch is a cluster.  Gamma-through-L1
+// launches are single blocks on the ring.
+template <typename TS, int D, int V, int kMode>
+int launch_layerwise_sched(int sched, void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
+                           const float *gq, const float *gk, float eps, int threads, int cluster,
+                           float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
+                           float *aux, cudaStream_t stream)
+{
+#define QKN_LW_LAUNCH(CL, SCHED)                                                               \
+    launch_layerwise_vpt<TS, D, V, CL, kMode, SCHED>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,  \
+                                                     threads, CL ? cluster : 1, inv_len_q,     \
+                                                     inv_len_k, plan_q, plan_k, aux, stream)
+    if constexpr (layerwise_gamma_regs<TS, V>()) {
+        if constexpr (kMode == kFused) {
+            if (sched == kSchedDirect)
+                return cluster > 1 ? QKN_LW_LAUNCH(true, kSchedDirect)
+                                   : QKN_LW_LAUNCH(false, kSchedDirect);
+            if constexpr (layerwise_overlap_type<TS>()) {
+                if (sched == kSchedOverlap)
+                    return cluster > 1 ? QKN_LW_LAUNCH(true, kSchedOverlap)
+                                       : QKN_LW_LAUNCH(false, kSchedOverlap);
+            }
+        }
+        if (cluster > 1) return QKN_LW_LAUNCH(true, kSchedRing);
+    }
+    return QKN_LW_LAUNCH(false, kSchedRing);
+#undef QKN_LW_LAUNCH
+}
+
 // Launch shape, chosen from measurements on B200 over the four storage types,
 // head_dim 64 to 256 and 40 to 72 heads:
 //  * the smallest cluster size CL (1, 2, 4 or 8 blocks, dividing the head
@@ -325,9 +363,12 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 //    registers (VPT * kVec <= 32) and the block within 576 threads;
 //  * the fewest such VPT, but at least 2: with one vector per thread the
 //    per-token work of a thread is too short for its fixed per-token cost;
-//  * on short inputs, fewer than 12 tokens per resident cluster, twice that
-//    VPT when gamma still fits: half the threads per block, about twice the
-//    resident blocks, so more tokens are under way at once.
+//  * on inputs of at most one block per SM (T times CL up to the SM count),
+//    that VPT with the direct schedule for fused launches: each block has one
+//    token, so there is nothing to prefetch and no ring;
+//  * on other short inputs, fewer than 12 tokens per resident cluster, twice
+//    that VPT when gamma still fits: half the threads per block, about twice
+//    the resident blocks, so more tokens are under way at once.
 // If no cluster size fits, one block per token with the fewest VPT within
 // 1024 threads, gamma read through L1 where it does not fit registers.
 // For fp32 and FP8 storage, a fused launch that keeps its VPT and is not
@@ -340,12 +381,6 @@ int launch_layerwise_vpt(void *qkv, int64_t T, int Hq, int Hk, int64_t row_strid
 constexpr int kLayerwiseMaxThreads = 576;
 constexpr int kLayerwiseShortTokens = 12;
 constexpr int kMaxCluster = 8;
-
-template <typename TS>
-constexpr bool layerwise_overlap_type()
-{
-    return Storage<TS>::kVec == 4 || Storage<TS>::kVec == 16;  // fp32, FP8
-}
 
 // Resident blocks per SM by the register file and the thread limit; the
 // shape rule's estimate (the launch itself queries the occupancy).
@@ -400,7 +435,7 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
             }
         }
     }
-    bool overlap = false;
+    int sched = kSchedRing;
     if (chosen != 0) {
         int dev = 0, rc;
         DeviceInfo info;
@@ -412,39 +447,34 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
         };
         const int ept = chosen * kVec;
         const bool can_double = 2 * ept <= 32 && vpt_ok(2 * chosen);
-        if (can_double && T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false)))
+        // The vectors per thread depend on the shape and T only, never on the
+        // mode, so the tensor-parallel steps sum exactly as the fused kernel.
+        bool doubled = false;
+        if (T * cluster <= info.sms) {
+            // At most one block per SM, each with one token: nothing to
+            // prefetch (measured on B200: T=1..64 gain 11-22%; at T=256, with
+            // SMs shared, the ring with twice the VPT is 7% faster).
+            if (kMode == kFused) sched = kSchedDirect;
+        } else if (can_double &&
+                   T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false))) {
             chosen *= 2;
-        else if (kMode == kFused && layerwise_overlap_type<TS>())
-            overlap = T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true));
+            doubled = true;
+        }
+        if (!doubled && kMode == kFused && layerwise_overlap_type<TS>() && sched == kSchedRing &&
+            T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true)))
+            sched = kSchedOverlap;
     }
     for (int vpt = 1; vpt <= kNV && chosen == 0; vpt *= 2)
         if (vpt_ok(vpt) && threads_for(1, vpt) <= 1024) chosen = vpt;
     if (chosen == 0) return QKN_ERR_UNSUPPORTED;
     const int threads = (int)(((heads / cluster * (kNV / chosen)) + 31) / 32 * 32);
-    constexpr bool kMayOverlap = kMode == kFused && layerwise_overlap_type<TS>();
 #define QKN_LW_CASE(V)                                                                         \
     case V:                                                                                    \
-        if constexpr (layerwise_vpt_ok<TS, D, V>()) {                                          \
-            if constexpr (layerwise_gamma_regs<TS, V>()) {                                     \
-                if constexpr (kMayOverlap) {                                                   \
-                    if (overlap && cluster > 1)                                                \
-                        return launch_layerwise_vpt<TS, D, V, true, kMode, true>(              \
-                            qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, cluster,         \
-                            inv_len_q, inv_len_k, plan_q, plan_k, aux, stream);                \
-                    if (overlap)                                                               \
-                        return launch_layerwise_vpt<TS, D, V, false, kMode, true>(             \
-                            qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, 1, inv_len_q,    \
-                            inv_len_k, plan_q, plan_k, aux, stream);                           \
-                }                                                                              \
-                if (cluster > 1)                                                               \
-                    return launch_layerwise_vpt<TS, D, V, true, kMode>(                        \
-                        qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, cluster, inv_len_q,  \
-                        inv_len_k, plan_q, plan_k, aux, stream);                               \
-            }                                                                                  \
-            return launch_layerwise_vpt<TS, D, V, false, kMode>(                               \
-                qkv, T, Hq, Hk, row_stride, gq, gk, eps, threads, 1, inv_len_q, inv_len_k,     \
-                plan_q, plan_k, aux, stream);                                                  \
-        }                                                                                      \
+        if constexpr (layerwise_vpt_ok<TS, D, V>())                                            \
+            return launch_layerwise_sched<TS, D, V, kMode>(sched, qkv, T, Hq, Hk, row_stride,   \
+                                                           gq, gk, eps, threads, cluster,      \
+                                                           inv_len_q, inv_len_k, plan_q,       \
+                                                           plan_k, aux, stream);               \
         break;
     switch (chosen) {
         QKN_LW_CASE(1)

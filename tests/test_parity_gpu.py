@@ -213,6 +213,26 @@ def test_layerwise_cluster_split(Hq, Hk, D, dtype, ns):
         assert np.array_equal(o, outs[0])
 
 
+@pytest.mark.parametrize("T", (1, 5, 37))
+@pytest.mark.parametrize("Hq,Hk,D,dtype", [(32, 8, 128, synth.BF16), (32, 8, 128, synth.FP8),
+                                           (112, 16, 256, synth.BF16), (256, 64, 256, synth.BF16)])
+def test_layerwise_decode_sizes(T, Hq, Hk, D, dtype):
+    """Decode-size inputs, at most one block per SM: the fused kernel loads each
+    token straight into registers (no staging ring), in single blocks or in
+    2- and 8-block clusters.  Every element against the oracle, the same bits
+    for every nshards, and for one rank the same bits as the two
+    tensor-parallel steps, which stage through the ring."""
+    c = synth.make_case(T, Hq, Hk, D, dtype=dtype, seed=90 + T + Hq, layerwise=True,
+                        scale="lognormal")
+    outs = [full_parity(c, "layerwise", n, what="decode T=%d n=%d" % (T, n))[0] for n in (1, 8)]
+    assert np.array_equal(outs[0], outs[1])
+    x, gq, gk = gu.to_device(c)
+    sums = qkn.qknorm_layerwise_partials(x, Hq, Hk, D)
+    qkn.qknorm_layerwise_apply(x, Hq, Hk, D, gq, gk, sums, Hq * D, Hk * D, c.eps)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.stored_bits(x), outs[0])
+
+
 @pytest.mark.parametrize("dtype", (synth.BF16, synth.FP8))
 def test_layerwise_gamma_through_l1(dtype):
     """129 heads of 256 (odd, so no cluster split): gamma cannot stay in
