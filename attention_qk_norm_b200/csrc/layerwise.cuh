@@ -153,9 +153,10 @@ enum LayerwiseSchedule { kSchedRing = 0, kSchedOverlap = 1, kSchedDirect = 2 };
 // [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
 // thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
 // per head), and thread l == 0 is the head's owner.  Dynamic shared memory
-// per block: kLayerwiseStages stages of this block's part of a token
-// (hc*D*sizeof(TS) bytes), two buffers of `heads` fp32 head partials
-// (alternating per token), then the two exchange barriers (CL > 1).  With
+// per block: the ring's kLayerwiseStages stages of this block's part of a
+// token (hc*D*sizeof(TS) bytes each; none with the direct schedule), two
+// buffers of `heads` fp32 head partials (alternating per token), then the
+// two exchange barriers (CL > 1).  With
 // CL = 1 the partials meet behind one block barrier per token; with CL > 1
 // each owner pushes its partial into every block of the cluster and each
 // block waits on its own barrier (see the exchange helpers above).

@@ -15,13 +15,15 @@
 // slice of gamma_q / gamma_k in registers for the whole launch.
 //
 // Layerwise (SwiftQK abstract; review key_machinery): a persistent block
-// walks tokens with a grid stride.  Each thread copies its vectors of
-// the next token into a two-stage shared-memory ring with cp.async while it
-// works on the current one.  The per-head partial sums of squares meet in
-// shared memory behind one barrier; then each warp, for the vectors (q, k)
-// its threads hold, forms every emulated shard's fp32 partial from that
-// shard's heads alone and combines the shard scalars, and every thread scales
-// its vectors, re-read from the ring, by the inverse RMS of its vector.
+// (or thread-block cluster, for tokens too wide for one block) walks tokens
+// with a grid stride.  Each thread copies its vectors of the next token into
+// a two-stage shared-memory ring with cp.async while it works on the current
+// one (at decode sizes it loads them straight into registers instead).  The
+// per-head partial sums of squares meet in shared memory behind one barrier
+// (across a cluster, on transaction barriers); then each warp, for the
+// vectors (q, k) its threads hold, forms every emulated shard's fp32 partial
+// from that shard's heads alone and combines the shard scalars, and every
+// thread scales its vectors by the inverse RMS of its vector.
 //
 // Both kernels are launched with programmatic dependent launch: they wait on
 // griddepcontrol.wait before their first global memory access, so a kernel
