@@ -675,6 +675,6 @@ int qknorm_wait_timeouts(unsigned int *count)
     return e == cudaSuccess ? QKN_OK : cuda_fail(e);
 }
 
-int qknorm_version(void) { return 103; }
+int qknorm_version(void) { return 104; }
 
 }  // extern "C"

@@ -18,9 +18,14 @@ a reported baseline, SM clocks sampled during the timed region, and a sweep
 over T and over the other workloads (GQA fused layout, layerwise with 1..8
 emulated shards, fp32 / head_dim 64..256 stress shapes).
 
-Under torchrun with N > 1 every rank runs the same per-GPU workload on its
-own GPU (weak scaling: tokens are independent, so no collective touches the
-data; NCCL carries only the barrier and the max of the timings).
+With N > 1 (``--gpus N``, started here under torch.distributed.run when no
+launcher set WORLD_SIZE, or under the caller's torchrun) every rank runs the
+same per-GPU workload on its own GPU (weak scaling: tokens are independent,
+so no collective touches the data; NCCL carries only the barrier and the max
+of the timings).  The line's ``tp`` entry times tensor-parallel layerwise
+QK-Norm with the layerwise workload's heads split over the N ranks: the
+scalar all-reduce exchange against the All-Gather baseline, per layer call.
+``--dry-run`` runs only the launch and the cross-rank steps, without a GPU.
 
 ``--impl reference`` times the float64 CPU oracle on the host cores instead
 (rank 0 only), on bounded samples of the same workload.
@@ -149,8 +154,19 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+def host_threads() -> int:
+    """Host cores this process may run on (a launcher's OMP_NUM_THREADS=1 per
+    rank does not shrink the CPU baseline)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 # ------------------------------------------------------------- distributed --
-def dist_init():
+def dist_init(use_gpu: bool = True):
+    """Join the process group of a torchrun launch (NCCL with a GPU per rank,
+    gloo on CPU); returns (rank, world size, local rank)."""
     import torch
     import torch.distributed as dist
     from datetime import timedelta
@@ -159,7 +175,7 @@ def dist_init():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and not dist.is_initialized():
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        backend = "nccl" if use_gpu and torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=timedelta(seconds=120),
@@ -343,6 +359,75 @@ def run_extras(device, l2, hbm_peak):
     return res
 
 
+# The layerwise workload's heads (32 query, 8 key/value, head_dim 128, bf16),
+# split by head over the ranks of a tensor-parallel group.
+TP_GLOBAL = dict(Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6)
+
+
+def time_eager_us(fn, bufs, world, iters=50, warm=5):
+    """Mean µs per call of ``fn(buf)`` over ``iters`` calls launched eagerly
+    (no graph: the calls hold collectives), rotating ``bufs``; CUDA events on
+    the current stream, max over ranks."""
+    import torch
+
+    for i in range(warm):
+        fn(bufs[i % len(bufs)])
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(iters):
+        fn(bufs[i % len(bufs)])
+    e.record()
+    torch.cuda.synchronize()
+    return max_over_ranks(s.elapsed_time(e) * 1e3 / iters, world)
+
+
+def run_tp(device, l2, world, rank, T_list=(1, 16, 256, 4096, 8192)):
+    """Tensor-parallel layerwise QK-Norm, the layerwise workload's heads split
+    over the ``world`` ranks: per layer call, the scalar exchange
+    (``qknorm_layerwise_tp``: partials, one all-reduce of 2T floats, scaling)
+    against the All-Gather baseline (``qknorm_layerwise_tp_allgather``)."""
+    import torch
+    import attention_qk_norm_b200 as qkn
+    from attention_qk_norm_b200 import synth
+
+    G = TP_GLOBAL
+    if G["Hq"] % world or G["Hk"] % world:
+        return {"world": world, "skipped": "the group size must divide 32 query and 8 key heads"}
+    hq, hk, D, eps = G["Hq"] // world, G["Hk"] // world, G["D"], G["eps"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2900)  # the same full-length weights on every rank
+    gq_full = 1.0 + 0.1 * torch.randn(G["Hq"] * D, generator=gen, device=device)
+    gk_full = 1.0 + 0.1 * torch.randn(G["Hk"] * D, generator=gen, device=device)
+    gq = gq_full[rank * hq * D:(rank + 1) * hq * D].contiguous()
+    gk = gk_full[rank * hk * D:(rank + 1) * hk * D].contiguous()
+    points = []
+    for T in T_list:
+        d = synth.make_case_torch(T, hq, hk, D, device=device, layerwise=True,
+                                  seed=2800 + T + 31 * rank)
+        one = d["qkv"].numel() * d["qkv"].element_size()
+        n = max(2, min(64, math.ceil(4 * l2 / max(1, one))))
+        bufs = [d["qkv"]] + [d["qkv"].clone() for _ in range(n - 1)]
+        ar = time_eager_us(lambda b: qkn.qknorm_layerwise_tp(b, hq, hk, D, gq, gk, eps), bufs,
+                           world)
+        ag = time_eager_us(lambda b: qkn.qknorm_layerwise_tp_allgather(b, hq, hk, D, gq_full,
+                                                                       gk_full, eps),
+                           bufs, world)
+        points.append({"T": T, "scalar_allreduce_us": round(ar, 3),
+                       "allgather_us": round(ag, 3),
+                       "allreduce_vs_allgather": round(ar / ag, 4)})
+        del bufs, d
+        torch.cuda.empty_cache()
+    return {"world": world, "heads_per_rank": {"q": hq, "kv": hk}, "head_dim": D,
+            "dtype": G["dtype"],
+            "workload": "layerwise QK-Norm of 32 query / 8 key heads x 128 split by head over "
+                        "%d rank(s), one layer call per step" % world,
+            "timing": "eager calls (they hold NCCL collectives), CUDA events, mean of 50, "
+                      "max over ranks",
+            "points": points}
+
+
 def e2e(w, device, steps, lanes=2):
     """Same metric through host buffers: per step a pinned-host -> device copy
     of the input, the C-ABI call, and a device -> pinned-host copy of the
@@ -399,7 +484,7 @@ def cpu_baseline(w, budget_s=10.0):
 
     c = synth.make_case(w["T"], w["Hq"], w["Hk"], w["D"], dtype=w["dtype"], seed=w["seed"],
                         eps=w["eps"])
-    threads = oracle.max_threads()
+    threads = host_threads()
     t0 = time.perf_counter()
     passes = 0
     while True:
@@ -441,8 +526,11 @@ def run_ours(args):
     full, rem = divmod(args.steps, GRAPH_STEPS)
     g_full = wl.graph(GRAPH_STEPS) if full else None
     g_rem = wl.graph(rem) if rem else None
-    if g_full is not None:
-        g_full.replay()
+    # Replay every graph once before timing: a graph's first replay uploads
+    # it to the device, which must not land inside the timed region.
+    for g in (g_full, g_rem):
+        if g is not None:
+            g.replay()
     torch.cuda.synchronize()
 
     sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
@@ -480,11 +568,12 @@ def run_ours(args):
     l2_note = ("rotating %d in-place buffers of %.1f MB (%.0f MB > 4x L2 %.0f MB)"
                % (len(wl.bufs), wl.buffer_bytes / 1e6, wl.buffer_bytes * len(wl.bufs) / 1e6,
                   l2 / 1e6))
-    extras = None
+    extras = tp = None
     if not args.no_extras:
         wl.free()
         torch.cuda.empty_cache()
         extras = run_extras(device, l2, hbm_peak)
+        tp = run_tp(device, l2, world, rank)
     barrier(world)
 
     if rank == 0:
@@ -515,6 +604,8 @@ def run_ours(args):
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
         if extras is not None:
             line["sweep"] = extras
+        if tp is not None:
+            line["tp"] = tp
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -534,7 +625,7 @@ def run_reference(args):
     w = HEADLINE
     c = synth.make_case(w["T"], w["Hq"], w["Hk"], w["D"], dtype=w["dtype"], seed=w["seed"],
                         eps=w["eps"])
-    threads = oracle.max_threads()
+    threads = host_threads()
 
     def step(n_tok, start):
         rows = [(start + i) % c.T for i in range(n_tok)]
@@ -621,17 +712,81 @@ def main(argv=None):
     ap.add_argument("--profile", choices=sorted(PROFILE_CASES),
                     help="only launch one workload's kernel (for ncu captures)")
     ap.add_argument("--profile-T", type=int, default=0)
+    ap.add_argument("--dry-run", action="store_true",
+                    help="check the rank launch and the cross-rank timing steps (barrier, max "
+                         "over ranks) without touching a GPU; rank 0 prints one JSON line")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.steps < 1:
         ap.error("--steps must be >= 1")
-    if args.profile:
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is not None and int(env_world) != args.gpus:
+        ap.error("--gpus %d disagrees with WORLD_SIZE=%s set by the launcher"
+                 % (args.gpus, env_world))
+    if env_world is None and args.gpus > 1:
+        # One process per GPU: start the N ranks here under torch.distributed.run.
+        if not args.dry_run:
+            import torch
+
+            have = torch.cuda.device_count()
+            if have < args.gpus:
+                ap.error("--gpus %d but only %d CUDA device(s) visible" % (args.gpus, have))
+        return self_launch(args.gpus, sys.argv[1:] if argv is None else list(argv))
+    if args.dry_run:
+        run_dry(args)
+    elif args.profile:
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
+    return 0
+
+
+def free_port() -> int:
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def self_launch(n: int, argv) -> int:
+    """Run this script as ``n`` ranks on this node under torch.distributed.run
+    (rendezvous on 127.0.0.1) with the same arguments; returns its exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_dry(args):
+    """The launch and cross-rank steps of a run, with no GPU work: every rank
+    joins the process group (gloo without CUDA), counts the ranks with a sum,
+    meets at the barrier and takes the max over ranks of a per-rank figure."""
+    rank, world, _ = dist_init(use_gpu=False)
+    count = world
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        t = torch.ones(1, dtype=torch.float64)
+        dist.all_reduce(t)
+        count = int(t.item())
+    barrier(world)
+    ms = max_over_ranks(1.0 + rank, world)
+    barrier(world)
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "impl": args.impl, "n_gpus": world,
+                          "ranks_counted": count, "max_over_ranks": ms, "steps": args.steps,
+                          "warmup": args.warmup}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -41,7 +41,9 @@
  * stay valid until the work on `stream` completes.  The library allocates
  * no memory and keeps no per-call state; calls are asynchronous and
  * stream-ordered, and the caller synchronises.  Entry points are safe to call
- * from several host threads.
+ * from several host threads, except that calls of qknorm_layerwise_noalloc
+ * share one scratch array per device and must be ordered on one stream (see
+ * there).
  *
  * Errors: each entry point returns QKN_OK or a negative qkn_status and
  * launches nothing when an argument is rejected.  Validation touches no CUDA
@@ -117,7 +119,10 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
  * memory and wait for them on transaction barriers; each such wait gives up
  * after 2 seconds, which can only happen if the GPU misbehaves, and is then
  * counted (see qknorm_wait_timeouts) while the kernel runs to its end with
- * wrong results.
+ * wrong results.  Such a call still returns QKN_OK, because the wait runs
+ * after the call has returned: a caller that must know reads
+ * qknorm_wait_timeouts before the call and again after synchronising with
+ * it, and treats the outputs of a call during which the count grew as wrong.
  */
 int qknorm_layerwise(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int64_t row_stride,
                      const float *gamma_q, const float *gamma_k, float eps, int nshards,
@@ -200,7 +205,8 @@ int qknorm_last_cuda_error(void);
 int qknorm_wait_timeouts(unsigned int *count);
 
 /* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3, 1.02 the
- * tensor-parallel layerwise steps, 1.03 qknorm_wait_timeouts). */
+ * tensor-parallel layerwise steps, 1.03 qknorm_wait_timeouts, 1.04
+ * qknorm_layerwise_noalloc and QKN_ERR_TOO_LARGE). */
 int qknorm_version(void);
 
 #ifdef __cplusplus

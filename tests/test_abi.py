@@ -49,7 +49,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.qknorm_version() == 103
+    assert lib.qknorm_version() == 104
     for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS, -8):
         s = lib.qknorm_status_string(code).decode()
         assert s and s != "unknown status"

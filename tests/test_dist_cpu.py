@@ -150,3 +150,33 @@ def test_algorithmic_bytes():
     assert bench.workload_bytes(w) == 2 * 4096 * 48 * 128 * 2 + 128 * 4
     lw = dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16")
     assert bench.workload_bytes(lw) == 2 * 8192 * 40 * 128 * 2 + 40 * 128 * 4
+
+
+def _bench(args, env_extra=None):
+    import subprocess
+    import sys
+
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, bench.__file__, *args], capture_output=True,
+                          text=True, env=env, timeout=300)
+
+
+def test_bench_gpus_flag_launches_that_many_ranks():
+    """``bench.py --gpus 2`` without a launcher starts two ranks itself; the
+    line reports both (gloo on CPU, --dry-run)."""
+    import json
+
+    r = _bench(["--gpus", "2", "--dry-run", "--steps", "4", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    assert lines[0]["n_gpus"] == 2 and lines[0]["ranks_counted"] == 2
+    assert lines[0]["max_over_ranks"] == 2.0  # rank 1's figure, seen by rank 0
+
+
+def test_bench_gpus_flag_must_match_the_launcher():
+    r = _bench(["--gpus", "2", "--dry-run"], {"WORLD_SIZE": "3", "RANK": "0"})
+    assert r.returncode != 0 and "disagrees" in r.stderr

@@ -74,6 +74,33 @@ def test_layerwise(T):
         assert np.array_equal(o, outs[0]), "layerwise output depends on nshards"
 
 
+@pytest.mark.parametrize("dtype", (synth.BF16, synth.FP16))
+def test_layerwise_config_largest_T_every_element(dtype):
+    """The layerwise workload at its largest T (8192), which takes the long-input
+    launch shape (two vectors per thread, 320-thread blocks, staging ring):
+    every element against the oracle for nshards 1 and 8, the same bits for
+    both."""
+    T = synth.LAYERWISE_T[-1]
+    c = synth.make_case(T, seed=synth.LAYERWISE_SEED + T, **dict(synth.LAYERWISE, dtype=dtype))
+    outs = [full_parity(c, "layerwise", n, what="layerwise %s T=%d n=%d" % (dtype, T, n))[0]
+            for n in (1, 8)]
+    assert np.array_equal(outs[0], outs[1]), "layerwise output depends on nshards"
+
+
+@pytest.mark.parametrize("D", synth.STRESS_D)
+def test_stress_layerwise_bf16_long_every_element(D):
+    """Stress layerwise (64 query / 8 key heads, lognormal scales over 1e-3..1e3,
+    zero and outlier rows) at 7200 tokens, long enough for the long-input
+    shape at every head_dim (single blocks at 64 and 128, 2-block clusters at
+    256): every element against the oracle, nshards 1 and 8 bit-identical."""
+    kw = dict(synth.STRESS, T=7200)
+    c = synth.make_case(D=D, dtype=synth.BF16, eps=1e-6, seed=synth.STRESS_SEED + 7 * D,
+                        layerwise=True, **kw)
+    outs = [full_parity(c, "layerwise", n, what="stress layerwise long D=%d n=%d" % (D, n))[0]
+            for n in (1, 8)]
+    assert np.array_equal(outs[0], outs[1])
+
+
 @pytest.mark.parametrize("dtype", synth.STRESS_DTYPES)
 @pytest.mark.parametrize("D", synth.STRESS_D)
 @pytest.mark.parametrize("eps", synth.STRESS_EPS)

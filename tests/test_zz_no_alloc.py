@@ -5,10 +5,12 @@ point keeps its intermediate per-token sums in a static array inside the
 library, so the caller passes only its own buffer and weights.
 
 The test calls it through the C ABI twice in a row, on two different inputs,
-and compares each result with the existing qknorm_layerwise entry point on
-the same input, within the parity tolerances of the other GPU tests.  The
-second call runs over the array the first one filled, so a result that
-depended on leftovers would show.  This file is collected last on purpose.
+and compares each result with the float64 oracle and with the existing
+qknorm_layerwise entry point on the same input, within the parity
+tolerances of the other GPU tests.  The second call runs over the array the
+first one filled, so a result that depended on leftovers would show.  The
+device counter of in-kernel waits that gave up must not move.  This file is
+collected last on purpose.
 """
 import ctypes
 
@@ -47,6 +49,8 @@ def test_noalloc_matches_layerwise_two_calls_in_a_row():
         synth.make_case(257, 64, 8, 64, dtype=synth.FP32, seed=302, layerwise=True,
                         scale="stress", zero_frac=0.02, outlier_frac=0.02),
     ]
+    torch.cuda.synchronize()
+    timeouts_before = qkn.wait_timeouts()
     for c in cases:
         mine, gq, gk = gu.to_device(c)
         ref = mine.clone()
@@ -55,7 +59,10 @@ def test_noalloc_matches_layerwise_two_calls_in_a_row():
         torch.cuda.synchronize()
         got, want = gu.stored_bits(mine), gu.stored_bits(ref)
         qk = (c.Hq + c.Hk) * c.D
+        oracle_want = gu.oracle_out(c, "layerwise", c.qkv, c.T)
+        gu.check(got, oracle_want, c.qkv, c.dtype, qk, "noalloc vs oracle T=%d" % c.T)
         gu.check(got, gu.as_f64(want, c.dtype), c.qkv, c.dtype, qk, "noalloc T=%d" % c.T)
+    assert qkn.wait_timeouts() == timeouts_before
 
 
 def test_noalloc_rejects_tokens_beyond_its_scratch():
