@@ -12,12 +12,15 @@ from ._binding import (  # noqa: F401
     QKN_FP16,
     QKN_FP32,
     QKNormError,
+    TPComm,
+    exchange_handles,
     load_library,
     qknorm_layerwise,
     qknorm_layerwise_apply,
     qknorm_layerwise_partials,
     qknorm_layerwise_tp,
     qknorm_layerwise_tp_allgather,
+    qknorm_layerwise_tp_p2p,
     qknorm_per_head,
     tp_allgather_full,
     tp_allreduce_,

@@ -63,6 +63,21 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.qknorm_version.restype = i32
         lib.qknorm_wait_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint)]
         lib.qknorm_wait_timeouts.restype = i32
+        lib.qknorm_tp_comm_create.argtypes = [i32, i32, i64, ctypes.c_double,
+                                              ctypes.POINTER(vp), vp]
+        lib.qknorm_tp_comm_create.restype = i32
+        lib.qknorm_tp_comm_connect.argtypes = [vp, vp]
+        lib.qknorm_tp_comm_connect.restype = i32
+        lib.qknorm_tp_comm_create_local.argtypes = [i32, i64, ctypes.c_double,
+                                                    ctypes.POINTER(vp)]
+        lib.qknorm_tp_comm_create_local.restype = i32
+        lib.qknorm_tp_comm_destroy.argtypes = [vp]
+        lib.qknorm_tp_comm_destroy.restype = i32
+        lib.qknorm_tp_comm_errors.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        lib.qknorm_tp_comm_errors.restype = i32
+        lib.qknorm_layerwise_tp_p2p.argtypes = [vp, vp, i32, i64, i32, i32, i32, i64, vp, vp, f32,
+                                                vp]
+        lib.qknorm_layerwise_tp_p2p.restype = i32
         if path == LIB_PATH:
             _lib = lib
         return lib
@@ -274,4 +289,128 @@ def qknorm_layerwise_tp_allgather(qkv, Hq, Hk, D, gamma_q_full, gamma_k_full, ep
     qknorm_layerwise(full, HQ, HK, D, gamma_q_full, gamma_k_full, eps)
     qkv[:, q0:k0] = full[:, rank * Hq * D:(rank + 1) * Hq * D]
     qkv[:, k0:k1] = full[:, HQ * D + rank * Hk * D:HQ * D + (rank + 1) * Hk * D]
+    return qkv
+
+
+# ------------------------------------------- in-kernel tensor-parallel exchange --
+IPC_HANDLE_BYTES = 64
+
+
+def exchange_handles(handle: bytes, group=None):
+    """Every rank's IPC handle, in rank order (one all-gather of host objects
+    over ``group``; just ``[handle]`` without an initialised process group)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return [handle]
+    out = [None] * dist.get_world_size(group)
+    dist.all_gather_object(out, handle, group=group)
+    return out
+
+
+class TPComm:
+    """Communicator of ``qknorm_layerwise_tp_p2p`` (see include/qknorm.h):
+    this rank's receive buffer and the other ranks' buffers mapped through
+    CUDA IPC, or a whole group emulated on one device (``TPComm.local``).
+
+    Create it on the device the rank runs on; ``close()`` (or garbage
+    collection) frees it, after a barrier over the group so that no peer is
+    still storing into this rank's buffer."""
+
+    def __init__(self, ptr, world, rank, nlocal, group=None):
+        self._ptr = ptr
+        self.world, self.rank, self.nlocal, self.group = world, rank, nlocal, group
+
+    @classmethod
+    def local(cls, world: int, max_tokens: int, timeout_s: float = 2.0) -> "TPComm":
+        """A group of ``world`` ranks on the current device, served by one
+        launch per call."""
+        ptr = ctypes.c_void_p()
+        _check("qknorm_tp_comm_create_local", load_library().qknorm_tp_comm_create_local(
+            int(world), int(max_tokens), float(timeout_s), ctypes.byref(ptr)))
+        return cls(ptr, int(world), 0, int(world))
+
+    @classmethod
+    def from_group(cls, max_tokens: int, group=None, timeout_s: float = 2.0) -> "TPComm":
+        """This process's rank of ``group`` (torch.distributed; one rank when it
+        is not initialised): create, all-gather the IPC handles, connect."""
+        import torch
+        import torch.distributed as dist
+
+        on = dist.is_available() and dist.is_initialized()
+        world = dist.get_world_size(group) if on else 1
+        rank = dist.get_rank(group) if on else 0
+        lib = load_library()
+        ptr = ctypes.c_void_p()
+        handle = (ctypes.c_char * IPC_HANDLE_BYTES)()
+        _check("qknorm_tp_comm_create", lib.qknorm_tp_comm_create(
+            world, rank, int(max_tokens), float(timeout_s), ctypes.byref(ptr), handle))
+        comm = cls(ptr, world, rank, 1, group)
+        handles = exchange_handles(bytes(handle), group)
+        if world > 1:
+            torch.cuda.synchronize()
+            dist.barrier(group)  # every rank's buffer exists before any opens it
+            joined = b"".join(handles)
+            _check("qknorm_tp_comm_connect", lib.qknorm_tp_comm_connect(ptr, joined))
+            dist.barrier(group)
+        return comm
+
+    def errors(self) -> int:
+        """Waits of this communicator that gave up since it was created."""
+        count = ctypes.c_uint(0)
+        _check("qknorm_tp_comm_errors",
+               load_library().qknorm_tp_comm_errors(self._ptr, ctypes.byref(count)))
+        return int(count.value)
+
+    def close(self):
+        if self._ptr is None:
+            return
+        import torch
+
+        torch.cuda.synchronize()
+        if self.nlocal == 1 and self.world > 1:
+            import torch.distributed as dist
+
+            if dist.is_available() and dist.is_initialized():
+                dist.barrier(self.group)
+        load_library().qknorm_tp_comm_destroy(self._ptr)
+        self._ptr = None
+
+    def __del__(self):
+        try:
+            if self._ptr is not None and (self.nlocal > 1 or self.world == 1):
+                load_library().qknorm_tp_comm_destroy(self._ptr)
+                self._ptr = None
+        except Exception:
+            pass
+
+
+def qknorm_layerwise_tp_p2p(comm: TPComm, qkv, Hq, Hk, D, gamma_q, gamma_k, eps, row_stride=None,
+                            stream=None):
+    """Tensor-parallel layerwise QK-Norm with the scalar exchange inside the
+    kernel, in place.  ``qkv``, ``gamma_q`` and ``gamma_k`` are this rank's
+    tensors, or lists with one entry per rank of a local communicator; each
+    rank holds ``Hq`` query and ``Hk`` key/value heads of every token."""
+    many = isinstance(qkv, (list, tuple))
+    xs = list(qkv) if many else [qkv]
+    gqs = list(gamma_q) if many else [gamma_q]
+    gks = list(gamma_k) if many else [gamma_k]
+    if not (len(xs) == len(gqs) == len(gks) == comm.nlocal):
+        raise ValueError("pass one qkv / gamma_q / gamma_k per rank the communicator serves (%d)"
+                         % comm.nlocal)
+    T, stride = None, None
+    for x, gq, gk in zip(xs, gqs, gks):
+        _device_check(x, gq, gk)
+        t, st = _rows(x, row_stride)
+        if (T, stride) not in ((None, None), (t, st)):
+            raise ValueError("every rank's buffer must have the same shape")
+        T, stride = t, st
+    vp = ctypes.c_void_p
+    arr_x = (vp * comm.nlocal)(*[x.data_ptr() for x in xs])
+    arr_q = (vp * comm.nlocal)(*[_gamma_ptr(g, "gamma_q") for g in gqs])
+    arr_k = (vp * comm.nlocal)(*[_gamma_ptr(g, "gamma_k") for g in gks])
+    rc = load_library().qknorm_layerwise_tp_p2p(
+        comm._ptr, arr_x, _dtype_code(xs[0]), T, Hq, Hk, D, stride, arr_q, arr_k, float(eps),
+        _stream_ptr(xs[0], stream))
+    _check("qknorm_layerwise_tp_p2p", rc)
     return qkv

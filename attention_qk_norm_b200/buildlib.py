@@ -18,6 +18,9 @@ SOURCES = [os.path.join(CSRC, "qknorm.cu")]
 HEADERS = [os.path.join(INCLUDE, "qknorm.h")] + sorted(
     os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh"))
 LIB_PATH = os.path.join(PKG, "libqknorm.so")
+# The tensor-parallel exchange protocol built for the host (tests only).
+TP_HOST_SOURCE = os.path.join(CSRC, "tp_exchange_host.cc")
+TP_HOST_LIB = os.path.join(PKG, "libqknorm_tp_host.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -65,5 +68,21 @@ def build(force: bool = False, extra_flags=(), out: str = LIB_PATH) -> str:
     return out
 
 
+def build_tp_host(force: bool = False) -> str:
+    """Compile the host build of the exchange protocol (tp_exchange.h) that
+    the CPU tests run with one process per rank."""
+    deps = [TP_HOST_SOURCE, os.path.join(CSRC, "tp_exchange.h")]
+    if (not force and os.path.exists(TP_HOST_LIB)
+            and all(os.path.getmtime(p) <= os.path.getmtime(TP_HOST_LIB) for p in deps)):
+        return TP_HOST_LIB
+    tmp = TP_HOST_LIB + ".%d.tmp" % os.getpid()
+    gxx = shutil.which("g++") or "g++"
+    subprocess.check_call([gxx, "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread", "-I", CSRC,
+                           TP_HOST_SOURCE, "-o", tmp])
+    os.replace(tmp, TP_HOST_LIB)
+    return TP_HOST_LIB
+
+
 if __name__ == "__main__":
     print(build(force=True))
+    print(build_tp_host(force=True))

@@ -8,6 +8,7 @@
 #include <cooperative_groups.h>
 
 #include "storage.cuh"
+#include "tp_exchange.h"
 
 namespace {
 
@@ -36,15 +37,21 @@ struct SumPlan {
 // butterflies below distance used/n form each shard's partial S_r from that
 // shard's heads only, and the remaining ones are the scalar combine of
 // S_0..S_{n-1}.  So the result does not depend on n, bit for bit.
+//
+// The butterflies at distances below per_shard and those above it are one
+// sequence of xor steps (distance 1, 2, 4, ... below `used`), unrolled here
+// with each step predicated on the warp-uniform plan.
 __device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p, int lane)
 {
     float v = 0.f;
-    if (lane < p.used)
-        for (int j = 0; j < p.per_lane; ++j) v += part[lane * p.per_lane + j];
-    for (int o = 1; o < p.per_shard; o <<= 1)  // rank-local partial S_r
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    for (int o = p.per_shard; o < p.used; o <<= 1)  // combine of the shard scalars
-        v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane < p.used) {  // used > 0 means per_lane >= 1
+        const float *q = part + lane * p.per_lane;
+        v = q[0];
+        for (int j = 1; j < p.per_lane; ++j) v += q[j];
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+        if (o < p.used) v += __shfl_xor_sync(0xffffffffu, v, o);
     return __shfl_sync(0xffffffffu, v, 0);
 }
 
@@ -55,27 +62,6 @@ __device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p,
 // the receiving block's barrier; a block's barrier phase completes once all
 // (Hq + Hk) partials of the token have landed and its own thread 0 has armed
 // the phase.  No cluster-wide barrier and no memory fence is on the token path.
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(arrivals)
-                 : "memory");
-}
-// Make the initialised barriers visible to the other blocks of the cluster.
-__device__ __forceinline__ void mbar_init_fence()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-// One arrival plus `bytes` expected transaction bytes for the current phase.
-__device__ __forceinline__ void mbar_arm(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 {
     uint32_t ok;
@@ -103,18 +89,6 @@ __device__ __forceinline__ void st_async_f32(uint32_t dst, float v, uint32_t bar
                  "r"(__float_as_uint(v)), "r"(bar)
                  : "memory");
 }
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Waits on a barrier give up after this long (they complete in microseconds
-// when the exchange works); each give-up is counted in g_wait_timeouts.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ unsigned int g_wait_timeouts;
-
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity)) return true;
@@ -133,7 +107,57 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 //              over all ranks and len_q, len_k the full vector lengths.
 // The mean S/L is formed as S * inv_len with inv_len = 1/L rounded to fp32
 // once per launch.
-enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
+//   kP2P:      tensor-parallel layerwise QK-Norm in one launch per rank: this
+//              rank's two sums of squares are stored into every rank's
+//              receive buffer (peer stores, see tp_exchange.h), the world
+//              ranks' sums of the token are read back from this rank's own
+//              buffer and combined in a fixed tree, and the rank's columns
+//              are scaled with the full lengths; x * gamma is formed before
+//              the exchange (the overlap schedule).
+enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2, kP2P = 3 };
+
+// The exchange of a kP2P launch (tp_exchange.h).
+struct P2PArgs {
+    uint64_t *recv[qkn_tp::kMaxWorld];  // every rank's receive buffer, as this GPU addresses it
+    unsigned int *errors;               // the group's count of waits that gave up
+    uint32_t *abort_tag;                // tag of a call in which a wait gave up
+    int64_t max_tokens;
+    uint64_t timeout_ns;
+    int world;
+    int rank;                           // rank of grid row 0 (blockIdx.y adds to it)
+    uint32_t parity, tag;
+};
+
+// 64-bit relaxed accesses at system scope: a peer's stores over NVLink and
+// this GPU's polls of them.  Each is single-copy atomic (naturally aligned).
+__device__ __forceinline__ void st_relaxed_sys_u64(uint64_t *p, uint64_t v)
+{
+    asm volatile("st.relaxed.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_relaxed_sys_u64(const uint64_t *p)
+{
+    uint64_t v;
+    asm volatile("ld.relaxed.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Element i of a small pointer array held in kernel parameters, with a
+// compile-time index on every access (no copy of the array to local memory).
+template <typename P, int N>
+__device__ __forceinline__ P pick(const P (&a)[N], int i)
+{
+    P r = a[0];
+#pragma unroll
+    for (int j = 1; j < N; ++j)
+        if (j == i) r = a[j];
+    return r;
+}
 
 // How a launch moves each token through its block.
 //   kSchedRing:    a two-stage cp.async ring in shared memory (the next token
@@ -165,7 +189,7 @@ __device__ __forceinline__ void
 layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                  const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
                  float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
-                 float *__restrict__ aux)
+                 float *__restrict__ aux, const P2PArgs *p2p = nullptr)
 {
     using S = Storage<TS>;
     using V = typename S::Vec;
@@ -210,6 +234,14 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
 
     pdl_wait_then_release();
+    // kP2P: lane r of a warp stores to, and polls the slot of, rank r.
+    uint64_t *peer_buf = nullptr;
+    const uint64_t *own_buf = nullptr;
+    bool gave_up = false;
+    if constexpr (kMode == kP2P) {
+        peer_buf = pick(p2p->recv, lane);
+        own_buf = pick(p2p->recv, p2p->rank + (int)blockIdx.y);
+    }
     // This thread's head weights (the partials step has none).
     const float *gb = gamma_q;
     if (kMode != kPartials && active)
@@ -226,22 +258,30 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
             for (int e = 0; e < kVec; ++e) g[v * kVec + e] = t4[e];
         }
     }
-    const int64_t col0 = (int64_t)h * D;          // in the token row
-    const int scol0 = (hl * D + l * kVec) * (int)sizeof(TS);  // in a stage
+    static_assert(kDirect || NST == 2, "the ring alternates two stages");
+    // Running addresses, advanced per token instead of recomputed: this
+    // thread's first vector of head h in the row of its current token (the
+    // row advances by step_bytes), and its vectors in the ring's two stages.
     // Each thread copies, and later reads, only its own vectors of a stage.
-    auto fetch = [&](int64_t tok, int st) {
+    const int64_t row_bytes = row_stride * (int64_t)sizeof(TS);
+    const int64_t step_bytes = stride * row_bytes;
+    const unsigned char *gcur = reinterpret_cast<const unsigned char *>(qkv) +
+                                (int64_t)h * D * (int64_t)sizeof(TS) + (int64_t)l * kVB +
+                                first * row_bytes;
+    const int scol0 = (hl * D + l * kVec) * (int)sizeof(TS);  // in a stage
+    const V *sp_cur = reinterpret_cast<const V *>(smem + scol0);
+    const V *sp_nxt = reinterpret_cast<const V *>(smem + span + scol0);
+    uint32_t ss_cur = smem_u32(sp_cur), ss_nxt = smem_u32(sp_nxt);
+    float *const part0 = part, *const part1 = part + heads;
+    auto fetch = [&](const unsigned char *src, int64_t tok, uint32_t dst) {
         if (active && tok < T) {
-            const V *src = reinterpret_cast<const V *>(qkv + tok * row_stride + col0);
-            V *dst = reinterpret_cast<V *>(smem + (size_t)st * span + scol0);
 #pragma unroll kUnroll
-            for (int v = 0; v < VPT; ++v) cp_async<kVB>(dst + v * kLPH, src + l + v * kLPH);
+            for (int v = 0; v < VPT; ++v)
+                cp_async_s(dst + (uint32_t)(v * kLPH * kVB), src + v * kLPH * kVB);
         }
         cp_async_commit();
     };
-    if constexpr (!kDirect) {
-#pragma unroll
-        for (int i = 0; i < NST - 1; ++i) fetch(first + (int64_t)i * stride, i);
-    }
+    if constexpr (!kDirect) fetch(gcur, first, ss_cur);
     if constexpr (kExchange) {
         if (threadIdx.x == 0) {
             mbar_init(&bar[0], 1);
@@ -255,22 +295,20 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
         // before the first remote write.
         cooperative_groups::this_cluster().sync();
     }
-    int st = 0;
     uint32_t it = 0;  // tokens this block has done; partials buffer it % 2
     bool timed_out = false;
     for (int64_t t = first; t < T; t += stride, ++it) {
-        const V *sp = nullptr;  // this thread's vectors of the token, staged (ring)
+        const V *sp = sp_cur;     // this thread's vectors of the token, staged (ring)
         V xr[kDirect ? VPT : 1];  // or in registers (direct)
         if constexpr (kDirect) {
-            const V *src = reinterpret_cast<const V *>(qkv + t * row_stride + col0);
+            const V *src = reinterpret_cast<const V *>(gcur);
 #pragma unroll
             for (int v = 0; v < VPT; ++v)
-                xr[v] = active ? load_stream(src + l + v * kLPH) : zero_vec<V>();
+                xr[v] = active ? load_stream(src + v * kLPH) : zero_vec<V>();
         } else {
             // Refill the stage this thread finished with on the previous token.
-            fetch(t + (int64_t)(NST - 1) * stride, (st + NST - 1) % NST);
-            cp_async_wait<NST - 1>();
-            sp = reinterpret_cast<const V *>(smem + (size_t)st * span + scol0);
+            fetch(gcur + step_bytes, t + stride, ss_nxt);
+            cp_async_wait<1>();
         }
         float rq = 0.f, rk = 0.f;
         float xg[kOverlap ? kEPT : 1];  // x * gamma, formed before the combine
@@ -302,7 +340,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
             // after it has finished reading this buffer.  (Every warp holds an
             // owner: its first thread.)
             const uint32_t pb = it & 1u;
-            float *pp = part + pb * heads;
+            float *pp = pb ? part1 : part0;
             if constexpr (kExchange) {
                 if (active && l == 0) {
                     const uint32_t dst = smem_u32(pp + h), b = smem_u32(&bar[pb]);
@@ -323,7 +361,65 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 if (active && l == 0) pp[h] = s;
                 __syncthreads();
             }
-            if constexpr (kMode == kPartials) {
+            if constexpr (kMode == kP2P) {
+                const int world = p2p->world;
+                const int me = p2p->rank + (int)blockIdx.y;
+                if (threadIdx.x < 32) {  // warp 0 sends this rank's two sums to every rank
+                    const float sq = warp_sumsq(pp, plan_q, lane);
+                    const float sk = warp_sumsq(pp + Hq, plan_k, lane);
+                    if (lane < world) {
+                        uint64_t *dst = peer_buf + qkn_tp::slot_word(p2p->parity, t, me, 0,
+                                                                     p2p->max_tokens, world);
+                        st_relaxed_sys_u64(dst, qkn_tp::pack(sq, p2p->tag));
+                        st_relaxed_sys_u64(dst + 1, qkn_tp::pack(sk, p2p->tag));
+                    }
+                }
+                if (need_q || need_k) {  // the world ranks' sums, from this rank's buffer
+                    float vq = 0.f, vk = 0.f;
+                    bool ok = true;
+                    if (lane < world) {
+                        const uint64_t *src =
+                            own_buf + qkn_tp::slot_word(p2p->parity, t, lane, 0, p2p->max_tokens,
+                                                        world);
+                        uint64_t wq = ld_relaxed_sys_u64(src), wk = ld_relaxed_sys_u64(src + 1);
+                        if (!gave_up &&
+                            !(qkn_tp::arrived(wq, p2p->tag) && qkn_tp::arrived(wk, p2p->tag))) {
+                            const uint64_t t0 = global_ns();
+                            for (;;) {
+                                wq = ld_relaxed_sys_u64(src);
+                                wk = ld_relaxed_sys_u64(src + 1);
+                                if (qkn_tp::arrived(wq, p2p->tag) && qkn_tp::arrived(wk, p2p->tag))
+                                    break;
+                                if (global_ns() - t0 > p2p->timeout_ns ||
+                                    ld_relaxed_gpu_u32(p2p->abort_tag) == p2p->tag) {
+                                    ok = false;
+                                    break;
+                                }
+                            }
+                        }
+                        vq = qkn_tp::value_of(wq);
+                        vk = qkn_tp::value_of(wk);
+                    }
+                    if (__any_sync(0xffffffffu, !ok) && !gave_up) {
+                        // Count it, tell the other blocks, and wait no more in
+                        // this launch (its outputs are wrong from here on).
+                        gave_up = true;
+                        if (lane == 0) {
+                            atomicAdd(p2p->errors, 1u);
+                            atomicAdd(&g_wait_timeouts, 1u);
+                            atomicExch(p2p->abort_tag, p2p->tag);
+                        }
+                    }
+                    for (int d = 1; d < world; d <<= 1) {  // fixed rank tree, tp_exchange.h
+                        vq += __shfl_xor_sync(0xffffffffu, vq, d);
+                        vk += __shfl_xor_sync(0xffffffffu, vk, d);
+                    }
+                    vq = __shfl_sync(0xffffffffu, vq, 0);
+                    vk = __shfl_sync(0xffffffffu, vk, 0);
+                    if (need_q) rq = rsqrtf(vq * inv_len_q + eps);
+                    if (need_k) rk = rsqrtf(vk * inv_len_k + eps);
+                }
+            } else if constexpr (kMode == kPartials) {
                 // One warp of the cluster's first block writes this rank's sums.
                 if (threadIdx.x < 32 && crank == 0) {
                     const float sq = warp_sumsq(pp, plan_q, lane);
@@ -340,7 +436,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
         }
         if (kMode != kPartials && active) {
             const float rinv = h < Hq ? rq : rk;
-            V *p = reinterpret_cast<V *>(qkv + t * row_stride + col0);
+            V *p = reinterpret_cast<V *>(const_cast<unsigned char *>(gcur));
 #pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float o[kVec];
@@ -362,10 +458,18 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) o[e] = f[e] * gv[e] * rinv;
                 }
-                store_stream(p + l + v * kLPH, S::pack(o));
+                store_stream(p + v * kLPH, S::pack(o));
             }
         }
-        if constexpr (!kDirect) st = (st + 1 == NST) ? 0 : st + 1;
+        gcur += step_bytes;
+        if constexpr (!kDirect) {
+            const V *tp = sp_cur;
+            sp_cur = sp_nxt;
+            sp_nxt = tp;
+            const uint32_t ts = ss_cur;
+            ss_cur = ss_nxt;
+            ss_nxt = ts;
+        }
     }
     cp_async_wait<0>();
     // No block leaves while a partner could still write into it.
@@ -418,6 +522,31 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kSched>(
         qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
         aux);
+}
+
+// Pointers of the ranks one kP2P launch serves: one (a rank on its own GPU)
+// or every rank of a group emulated on one GPU (grid row y serves rank
+// p2p.rank + y).
+struct TPRankPtrs {
+    void *qkv[qkn_tp::kMaxWorld];
+    const float *gamma_q[qkn_tp::kMaxWorld];
+    const float *gamma_k[qkn_tp::kMaxWorld];
+};
+
+// Tensor-parallel layerwise QK-Norm with the exchange inside the kernel
+// (kP2P, overlap schedule, one block per token, gamma in registers).  All
+// blocks of the launch must be resident together (a cooperative launch),
+// since blocks of one token on different ranks wait for one another.
+template <typename TS, int D, int VPT>
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, true)))
+qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, int Hk,
+                        float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                        SumPlan plan_k, P2PArgs p2p)
+{
+    const int y = (int)blockIdx.y;
+    layerwise_tokens<TS, D, VPT, true, false, kP2P, kSchedOverlap>(
+        static_cast<TS *>(pick(ptrs.qkv, y)), row_stride, T, Hq, Hk, pick(ptrs.gamma_q, y),
+        pick(ptrs.gamma_k, y), eps, inv_len_q, inv_len_k, plan_q, plan_k, nullptr, &p2p);
 }
 
 // Gamma read through L1 (tokens too wide for registers; one block per token,

@@ -233,10 +233,51 @@ int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, 
                       gk, eps, (uint32_t)q_blocks);
 }
 
+template <typename TS, int D, bool kHasK>
+int launch_per_head_bulk(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
+                         const float *gq, const float *gk, float eps, cudaStream_t stream)
+{
+    using B = BulkShape<TS, D>;
+    auto kern = qkn_per_head_bulk_kernel<TS, D, kHasK>;
+    static KernelCache kc;
+    int dev = 0, per_sm = 0, rc;
+    DeviceInfo info;
+    if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
+    if (B::kSmemBytes > info.smem_optin) return QKN_ERR_UNSUPPORTED;
+    if ((rc = resident_blocks(kern, kc, dev, info, kBulkThreads, B::kSmemBytes, &per_sm)) != QKN_OK)
+        return rc;
+    if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
+    const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
+    const uint64_t nchunks = (rows + B::kChunkRows - 1) / B::kChunkRows;
+    const uint64_t cap = (uint64_t)info.sms * per_sm;
+    const uint64_t grid = nchunks < cap ? nchunks : cap;
+    return launch_pdl(kern, (unsigned)grid, kBulkThreads, B::kSmemBytes, stream, 1u,
+                      static_cast<TS *>(qkv), row_stride, T, (uint32_t)(Hq + Hk), (uint32_t)Hq, gq,
+                      gk, eps, nchunks);
+}
+
+// Inputs of at least this many Q/K bytes take the bulk-staged kernel.
+#ifndef QKN_PH_BULK_MIN_BYTES
+#define QKN_PH_BULK_MIN_BYTES (1ll << 62)
+#endif
+#ifndef QKN_PH_BULK_MIN_BYTES_FP8
+#define QKN_PH_BULK_MIN_BYTES_FP8 (1ll << 62)
+#endif
+
 template <typename TS, int D>
 int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                     const float *gk, float eps, cudaStream_t stream)
 {
+    const int64_t qk_bytes = T * (int64_t)(Hq + Hk) * D * (int64_t)sizeof(TS);
+    const int64_t bulk_min =
+        Storage<TS>::kVec == 16 ? (int64_t)QKN_PH_BULK_MIN_BYTES_FP8 : (int64_t)QKN_PH_BULK_MIN_BYTES;
+    if (qk_bytes >= bulk_min) {
+        if (Hq > 0 && Hk > 0)
+            return launch_per_head_bulk<TS, D, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
+                                                     stream);
+        return launch_per_head_bulk<TS, D, false>(qkv, T, Hq, Hk, row_stride, Hq > 0 ? gq : gk,
+                                                  nullptr, eps, stream);
+    }
     if (Hq > 0 && Hk > 0) {
         if constexpr (Storage<TS>::kVec == 16)  // FP8
             return launch_per_head_k<TS, D, false, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
@@ -512,6 +553,83 @@ int dispatch(int dtype, int D, Args... args)
 #undef QKN_BY_D
 }
 
+// ---------------------------------------- tensor-parallel exchange, P2P --
+// Launch shape of the in-kernel exchange: one block per token (no cluster),
+// gamma in registers, the fewest vectors per thread (at least 2) within 576
+// threads.
+template <typename TS, int D, int VPT>
+int launch_tp_vpt(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
+                  int64_t row_stride, float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
+                  SumPlan plan_k, const P2PArgs &p2p, int threads, cudaStream_t stream)
+{
+    auto kern = qkn_layerwise_tp_kernel<TS, D, VPT>;
+    static KernelCache kc;
+    const int heads = Hq + Hk;
+    const size_t span = (size_t)heads * D * sizeof(TS);
+    const size_t smem = kLayerwiseStages * span + (size_t)2 * heads * sizeof(float);
+    int dev = 0, per_sm = 0, rc;
+    DeviceInfo info;
+    if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
+    if (smem > (size_t)info.smem_optin) return QKN_ERR_UNSUPPORTED;
+    if ((rc = resident_blocks(kern, kc, dev, info, threads, smem, &per_sm)) != QKN_OK) return rc;
+    // Every block of every rank served here is resident at once.
+    const int64_t per_rank = (int64_t)info.sms * per_sm / nlocal;
+    if (per_rank < 1) return QKN_ERR_UNSUPPORTED;
+    const int64_t blocks = T < per_rank ? T : per_rank;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks, (unsigned)nlocal);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ptrs, row_stride, T, Hq, Hk, eps, inv_len_q,
+                                       inv_len_k, plan_q, plan_k, p2p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
+}
+
+struct LayerwiseTP {
+    template <typename TS, int D>
+    static int run(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
+                   int64_t row_stride, float eps, float len_q, float len_k, const P2PArgs &p2p,
+                   cudaStream_t stream)
+    {
+        constexpr int kVec = Storage<TS>::kVec;
+        constexpr int kNV = D / kVec;
+        const int heads = Hq + Hk;
+        int vpt = 0;
+        for (int v = 2; v * kVec <= 32 && vpt == 0; v *= 2)
+            if (v <= kNV && kNV % v == 0 && kNV / v <= 32 &&
+                (heads * (kNV / v) + 31) / 32 * 32 <= kLayerwiseMaxThreads)
+                vpt = v;
+        if (vpt == 0) return QKN_ERR_UNSUPPORTED;
+        const int threads = (heads * (kNV / vpt) + 31) / 32 * 32;
+        const float inv_len_q = Hq > 0 ? 1.0f / len_q : 0.f;
+        const float inv_len_k = Hk > 0 ? 1.0f / len_k : 0.f;
+        const SumPlan plan_q = sum_plan(Hq, 1), plan_k = sum_plan(Hk, 1);
+#define QKN_TP_CASE(V)                                                                         \
+    case V:                                                                                    \
+        if constexpr (layerwise_vpt_ok<TS, D, V>() && layerwise_gamma_regs<TS, V>())           \
+            return launch_tp_vpt<TS, D, V>(ptrs, nlocal, T, Hq, Hk, row_stride, eps,           \
+                                           inv_len_q, inv_len_k, plan_q, plan_k, p2p,          \
+                                           threads, stream);                                   \
+        break;
+        switch (vpt) {
+            QKN_TP_CASE(2)
+            QKN_TP_CASE(4)
+            QKN_TP_CASE(8)
+        default:
+            break;
+        }
+#undef QKN_TP_CASE
+        return QKN_ERR_UNSUPPORTED;
+    }
+};
+
 struct PerHead {
     template <typename TS, int D, typename... A>
     static int run(A... a) { return launch_per_head<TS, D>(a...); }
@@ -562,6 +680,87 @@ int noalloc_scratch(float **out)
         g_noalloc_ptr[dev] = static_cast<float *>(p);
     }
     *out = g_noalloc_ptr[dev];
+    return QKN_OK;
+}
+}  // namespace
+
+// The communicator of qknorm_layerwise_tp_p2p (see include/qknorm.h).
+struct qkn_tp_comm {
+    int world = 0, rank = 0, nlocal = 0, device = -1;
+    int64_t max_tokens = 0;
+    uint64_t calls = 0;
+    uint64_t timeout_ns = 0;
+    bool connected = false;
+    uint64_t *own[qkn_tp::kMaxWorld] = {};   // buffers this communicator allocated
+    uint64_t *recv[qkn_tp::kMaxWorld] = {};  // every rank's buffer, as this device addresses it
+    bool opened[qkn_tp::kMaxWorld] = {};     // recv[r] is an IPC mapping to close
+    unsigned int *errors = nullptr;          // device counter of waits that gave up
+    uint32_t *abort_tag = nullptr;
+};
+
+namespace {
+constexpr size_t kTPTailBytes = 256;  // the counter and the abort tag, after own[0]'s slots
+
+bool tp_world_ok(int world) { return world == 1 || world == 2 || world == 4 || world == 8; }
+
+// Allocate and zero `n` receive buffers on the current device.
+int tp_alloc(qkn_tp_comm *c, int n)
+{
+    const size_t bytes = qkn_tp::buffer_words(c->max_tokens, c->world) * sizeof(uint64_t);
+    for (int i = 0; i < n; ++i) {
+        void *p = nullptr;
+        cudaError_t e = cudaMalloc(&p, bytes + (i == 0 ? kTPTailBytes : 0));
+        if (e == cudaSuccess) e = cudaMemset(p, 0, bytes + (i == 0 ? kTPTailBytes : 0));
+        if (e != cudaSuccess) {
+            if (p != nullptr) cudaFree(p);
+            return cuda_fail(e);
+        }
+        c->own[i] = static_cast<uint64_t *>(p);
+    }
+    unsigned char *tail = reinterpret_cast<unsigned char *>(c->own[0]) + bytes;
+    c->errors = reinterpret_cast<unsigned int *>(tail);
+    c->abort_tag = reinterpret_cast<uint32_t *>(tail + 128);
+    return QKN_OK;
+}
+
+void tp_free(qkn_tp_comm *c)
+{
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (c->device >= 0) cudaSetDevice(c->device);
+    for (int r = 0; r < qkn_tp::kMaxWorld; ++r)
+        if (c->opened[r]) cudaIpcCloseMemHandle(c->recv[r]);
+    for (int i = 0; i < qkn_tp::kMaxWorld; ++i)
+        if (c->own[i] != nullptr) cudaFree(c->own[i]);
+    if (prev >= 0) cudaSetDevice(prev);
+    delete c;
+}
+
+int tp_create(int world, int rank, int nlocal, int64_t max_tokens, double timeout_s,
+              qkn_tp_comm **out)
+{
+    if (out == nullptr) return QKN_ERR_NULL;
+    *out = nullptr;
+    if (!tp_world_ok(world) || rank < 0 || rank >= world) return QKN_ERR_NSHARDS;
+    if (max_tokens < 1 || max_tokens > (int64_t)1 << 24) return QKN_ERR_SHAPE;
+    if (!(timeout_s > 0.0) || timeout_s > 3600.0) return QKN_ERR_SHAPE;
+    qkn_tp_comm *c = new qkn_tp_comm;
+    c->world = world;
+    c->rank = rank;
+    c->nlocal = nlocal;
+    c->max_tokens = max_tokens;
+    c->timeout_ns = (uint64_t)(timeout_s * 1e9);
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e != cudaSuccess) {
+        delete c;
+        return cuda_fail(e);
+    }
+    const int rc = tp_alloc(c, nlocal);
+    if (rc != QKN_OK) {
+        tp_free(c);
+        return rc;
+    }
+    *out = c;
     return QKN_OK;
 }
 }  // namespace
@@ -649,6 +848,112 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
                                     scratch);
 }
 
+int qknorm_tp_comm_create(int world, int rank, int64_t max_tokens, double timeout_s,
+                          qkn_tp_comm **comm, void *ipc_handle)
+{
+    if (ipc_handle == nullptr) return QKN_ERR_NULL;
+    int rc = tp_create(world, rank, 1, max_tokens, timeout_s, comm);
+    if (rc != QKN_OK) return rc;
+    qkn_tp_comm *c = *comm;
+    c->recv[rank] = c->own[0];
+    const cudaError_t e =
+        cudaIpcGetMemHandle(static_cast<cudaIpcMemHandle_t *>(ipc_handle), c->own[0]);
+    if (e != cudaSuccess) {
+        tp_free(c);
+        *comm = nullptr;
+        return cuda_fail(e);
+    }
+    if (world == 1) c->connected = true;
+    return QKN_OK;
+}
+
+int qknorm_tp_comm_connect(qkn_tp_comm *comm, const void *ipc_handles)
+{
+    if (comm == nullptr || ipc_handles == nullptr) return QKN_ERR_NULL;
+    if (comm->nlocal != 1) return QKN_ERR_UNSUPPORTED;
+    if (comm->connected) return QKN_OK;
+    const cudaIpcMemHandle_t *h = static_cast<const cudaIpcMemHandle_t *>(ipc_handles);
+    for (int r = 0; r < comm->world; ++r) {
+        if (r == comm->rank) continue;
+        void *p = nullptr;
+        const cudaError_t e = cudaIpcOpenMemHandle(&p, h[r], cudaIpcMemLazyEnablePeerAccess);
+        if (e != cudaSuccess) return cuda_fail(e);
+        comm->recv[r] = static_cast<uint64_t *>(p);
+        comm->opened[r] = true;
+    }
+    comm->connected = true;
+    return QKN_OK;
+}
+
+int qknorm_tp_comm_create_local(int world, int64_t max_tokens, double timeout_s,
+                                qkn_tp_comm **comm)
+{
+    const int rc = tp_create(world, 0, world, max_tokens, timeout_s, comm);
+    if (rc != QKN_OK) return rc;
+    for (int r = 0; r < world; ++r) (*comm)->recv[r] = (*comm)->own[r];
+    (*comm)->connected = true;
+    return QKN_OK;
+}
+
+int qknorm_tp_comm_destroy(qkn_tp_comm *comm)
+{
+    if (comm == nullptr) return QKN_ERR_NULL;
+    tp_free(comm);
+    return QKN_OK;
+}
+
+int qknorm_tp_comm_errors(qkn_tp_comm *comm, unsigned int *count)
+{
+    if (comm == nullptr || count == nullptr) return QKN_ERR_NULL;
+    const cudaError_t e = cudaMemcpy(count, comm->errors, sizeof(unsigned int),
+                                     cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? QKN_OK : cuda_fail(e);
+}
+
+int qknorm_layerwise_tp_p2p(qkn_tp_comm *comm, void *const *qkv, int dtype, int64_t T, int Hq,
+                            int Hk, int D, int64_t row_stride, const float *const *gamma_q,
+                            const float *const *gamma_k, float eps, void *stream)
+{
+    if (comm == nullptr || qkv == nullptr || gamma_q == nullptr || gamma_k == nullptr)
+        return QKN_ERR_NULL;
+    bool done = false;
+    for (int i = 0; i < comm->nlocal; ++i) {
+        const int rc = validate(qkv[i], dtype, T, Hq, Hk, D, row_stride, gamma_q[i], gamma_k[i],
+                                eps, &done);
+        if (rc != QKN_OK) return rc;
+    }
+    if (T > comm->max_tokens) return QKN_ERR_TOO_LARGE;
+    if (done) return QKN_OK;
+    if (!comm->connected) return QKN_ERR_UNSUPPORTED;
+    if (comm->calls >= qkn_tp::kMaxCalls) return QKN_ERR_TOO_LARGE;
+    int dev = -1;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev != comm->device) return QKN_ERR_UNSUPPORTED;
+    TPRankPtrs ptrs = {};
+    for (int i = 0; i < comm->nlocal; ++i) {
+        ptrs.qkv[i] = qkv[i];
+        ptrs.gamma_q[i] = gamma_q[i];
+        ptrs.gamma_k[i] = gamma_k[i];
+    }
+    P2PArgs a = {};
+    for (int r = 0; r < comm->world; ++r) a.recv[r] = comm->recv[r];
+    a.errors = comm->errors;
+    a.abort_tag = comm->abort_tag;
+    a.max_tokens = comm->max_tokens;
+    a.timeout_ns = comm->timeout_ns;
+    a.world = comm->world;
+    a.rank = comm->rank;
+    a.parity = qkn_tp::call_parity(comm->calls);
+    a.tag = qkn_tp::call_tag(comm->calls);
+    const float len_q = (float)((int64_t)Hq * D * comm->world);
+    const float len_k = (float)((int64_t)Hk * D * comm->world);
+    const int rc = dispatch<LayerwiseTP>(dtype, D, ptrs, comm->nlocal, T, Hq, Hk, row_stride, eps,
+                                         len_q, len_k, a, static_cast<cudaStream_t>(stream));
+    if (rc == QKN_OK) ++comm->calls;
+    return rc;
+}
+
 const char *qknorm_status_string(int status)
 {
     switch (status) {
@@ -675,6 +980,6 @@ int qknorm_wait_timeouts(unsigned int *count)
     return e == cudaSuccess ? QKN_OK : cuda_fail(e);
 }
 
-int qknorm_version(void) { return 104; }
+int qknorm_version(void) { return 105; }
 
 }  // extern "C"

@@ -114,21 +114,23 @@ class ClockSampler:
         self.proc = None
         self.out = None
 
-    def start(self):
+    def start(self, settle_s: float = 0.3):
+        """Start sampling; returns at once, and ``settle_s`` seconds are left
+        for nvidia-smi to come up (the caller keeps the GPU busy meanwhile)."""
+        self.ready_at = time.perf_counter() + settle_s
         try:
             self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
         except Exception:
             self.proc = None
 
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.15)
+        time.sleep(max(0.15, self.ready_at - time.perf_counter()))
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -519,24 +521,32 @@ def run_ours(args):
     hbm_peak, peak_kind = peaks()
     w = dict(HEADLINE)
     wl = Workload(w, device, l2)
-
-    for _ in range(args.warmup):
-        wl.launch()
-    torch.cuda.synchronize()
     full, rem = divmod(args.steps, GRAPH_STEPS)
     g_full = wl.graph(GRAPH_STEPS) if full else None
     g_rem = wl.graph(rem) if rem else None
-    # Replay every graph once before timing: a graph's first replay uploads
-    # it to the device, which must not land inside the timed region.
+    # Replay every graph once: a graph's first replay uploads it to the
+    # device, which must not land inside the timed region.
     for g in (g_full, g_rem):
         if g is not None:
             g.replay()
     torch.cuda.synchronize()
 
+    # The clock sampler starts first; while it comes up the GPU replays a
+    # warm-up graph (untimed), so that it does not idle, and drop its clocks,
+    # right before the timed region.  Then the W warm-up steps.
     sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                            if world == 1 else local)
+    g_warm = wl.graph(GRAPH_STEPS)
     if rank == 0:
         sampler.start()
+    settle_until = time.perf_counter() + 0.3
+    while time.perf_counter() < settle_until:
+        g_warm.replay()
+        torch.cuda.synchronize()
+    del g_warm
+    barrier(world)
+    for _ in range(args.warmup):
+        wl.launch()
     barrier(world)
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -662,6 +672,8 @@ def run_reference(args):
 
 PROFILE_CASES = {
     "per_head": dict(HEADLINE),
+    "per_head_h16": dict(HEADLINE, Hq=16),
+    "per_head_h32": dict(HEADLINE, Hq=32),
     "gqa": dict(kind="per_head", T=16384, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6, nshards=1,
                 scale="lognormal", seed=1002),
     "layerwise": dict(kind="layerwise", T=8192, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
@@ -683,7 +695,10 @@ PROFILE_CASES = {
 
 def run_profile(args):
     """A few plain launches of one workload, for a profiler to capture: no
-    graphs, no timing, no sweep.  ``--profile-T`` overrides the token count."""
+    graphs, no timing, no sweep.  ``--profile-T`` overrides the token count.
+    Launches rotate over copies of the input totalling more than 4x L2, as in
+    the timed runs, so a capture without cache flushes sees steady-state DRAM
+    traffic."""
     import torch
 
     w = dict(PROFILE_CASES[args.profile])
@@ -691,7 +706,9 @@ def run_profile(args):
         w["T"] = args.profile_T
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(device)
-    wl = Workload(w, device, l2_bytes=0)  # one buffer; profilers flush caches themselves
+    props = torch.cuda.get_device_properties(device)
+    wl = Workload(w, device, l2_bytes=int(getattr(props, "L2_cache_size", 126 << 20)),
+                  max_bytes=4 << 30)
     for _ in range(args.warmup + args.steps):
         wl.launch()
     torch.cuda.synchronize()

@@ -191,6 +191,83 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
                              int64_t row_stride, const float *gamma_q, const float *gamma_k,
                              float eps, void *stream);
 
+/*
+ * Tensor-parallel layerwise QK-Norm with the scalar exchange inside the
+ * kernel, as SwiftQK does it.  Sources: the SwiftQK abstract (ranks exchange
+ * only scalar statistics instead of gathering the hidden vectors) and the
+ * SwiftQK review (key_machinery: warp 0 of each block writes the partial sums
+ * to the peers' buffers and waits on flags, and the weight multiplication
+ * overlaps the exchange; major_comments[0]: the wait must not deadlock;
+ * major_comments[2]: the ordering of flag and payload).
+ *
+ * A group of `world` ranks (1, 2, 4 or 8) holds every token; each rank holds
+ * Hq query and Hk key/value heads of it in the fused layout described at the
+ * top (its share, split by head).  One call per rank, with the same T and the
+ * same sequence of calls on every rank: each block stages a token, forms its
+ * heads' fp32 partial sums of squares and the rank's two sums (q, k) with the
+ * fixed tree of qknorm_layerwise, stores them into every rank's receive
+ * buffer, forms x * gamma while the other ranks' sums arrive, reads the world
+ * ranks' sums back from its own buffer, combines them in a fixed pairwise
+ * tree in rank order (every rank gets the same bits), and scales its columns
+ * in place by 1/sqrt(S / L + eps) with L = Hq*D*world (q) or Hk*D*world (k).
+ * gamma_q / gamma_k are this rank's slices (Hq*D and Hk*D floats).
+ *
+ * The exchange: each of a rank's partial sums travels as one 8-byte word
+ * {fp32 value, 32-bit call tag}, written with a single peer store (no
+ * multicast, no collective library) into the receive buffer of each rank, which
+ * lives in that rank's device memory and is mapped into the others with CUDA
+ * IPC.  A reader polls its own buffer until every rank's word of the token
+ * carries the current call's tag.  Calls alternate between two halves of the
+ * buffer, so the buffer is never cleared between calls.
+ *
+ * Waits: the blocks of one token on different ranks wait for one another, so
+ * every block of a launch is made resident at once (a cooperative launch;
+ * it fails with QKN_ERR_CUDA rather than start partly), and blocks take
+ * tokens in the same order on every rank.  Each wait gives up after the
+ * communicator's time limit; the first give-up of a call is counted
+ * (qknorm_tp_comm_errors, and qknorm_wait_timeouts) and stops every other
+ * wait of that call on this rank, so a call whose peer never comes ends
+ * after about one time limit with wrong outputs instead of hanging.  Check
+ * qknorm_tp_comm_errors after synchronising to detect it.
+ *
+ * qknorm_tp_comm_create: set up this process's rank on the current device:
+ *   allocates its receive buffer (2 * max_tokens * world * 16 bytes plus 256,
+ *   zeroed; max_tokens in [1, 2^24]) and writes its CUDA IPC handle (64 bytes,
+ *   caller-owned) to ipc_handle.  timeout_s (0 < t <= 3600) is the time limit
+ *   of each wait.  Returns QKN_ERR_NSHARDS for a bad world or rank.
+ * qknorm_tp_comm_connect: ipc_handles holds the world ranks' handles in rank
+ *   order (world * 64 bytes, as exchanged by the caller, e.g. an all-gather);
+ *   opens the other ranks' buffers.  Every rank must be created before any
+ *   connects.  A world of 1 needs no connect.
+ * qknorm_tp_comm_create_local: a group of `world` ranks emulated on the
+ *   current device (all receive buffers local; no IPC); one call of
+ *   qknorm_layerwise_tp_p2p then serves every rank in one launch.
+ * qknorm_tp_comm_destroy: unmaps and frees.  Every rank must first have
+ *   finished its last call (synchronise, then meet at a barrier), since peers
+ *   store into this rank's buffer.
+ * qknorm_layerwise_tp_p2p: qkv, gamma_q and gamma_k are host arrays of device
+ *   pointers, one entry per rank the communicator serves (1, or world for a
+ *   local group, in rank order).  QKN_ERR_TOO_LARGE if T > max_tokens or the
+ *   communicator has made 2 * (2^32 - 2) calls; QKN_ERR_UNSUPPORTED if not
+ *   connected, the current device is not the communicator's, or the token is
+ *   too wide for one block of at most 576 threads with gamma in registers.
+ *   Other arguments and errors as qknorm_layerwise.
+ * qknorm_tp_comm_errors: waits of this communicator that gave up, since it was
+ *   created (a blocking copy; synchronise with the calls first).
+ */
+typedef struct qkn_tp_comm qkn_tp_comm;
+
+int qknorm_tp_comm_create(int world, int rank, int64_t max_tokens, double timeout_s,
+                          qkn_tp_comm **comm, void *ipc_handle);
+int qknorm_tp_comm_connect(qkn_tp_comm *comm, const void *ipc_handles);
+int qknorm_tp_comm_create_local(int world, int64_t max_tokens, double timeout_s,
+                                qkn_tp_comm **comm);
+int qknorm_tp_comm_destroy(qkn_tp_comm *comm);
+int qknorm_tp_comm_errors(qkn_tp_comm *comm, unsigned int *count);
+int qknorm_layerwise_tp_p2p(qkn_tp_comm *comm, void *const *qkv, int dtype, int64_t T, int Hq,
+                            int Hk, int D, int64_t row_stride, const float *const *gamma_q,
+                            const float *const *gamma_k, float eps, void *stream);
+
 /* Static English text for a qkn_status value (never NULL). */
 const char *qknorm_status_string(int status);
 
@@ -206,7 +283,8 @@ int qknorm_wait_timeouts(unsigned int *count);
 
 /* ABI version: 100 * major + minor (1.01 added QKN_FP16 and QKN_FP8_E4M3, 1.02 the
  * tensor-parallel layerwise steps, 1.03 qknorm_wait_timeouts, 1.04
- * qknorm_layerwise_noalloc and QKN_ERR_TOO_LARGE). */
+ * qknorm_layerwise_noalloc and QKN_ERR_TOO_LARGE, 1.05 the in-kernel
+ * tensor-parallel exchange: qknorm_tp_comm_* and qknorm_layerwise_tp_p2p). */
 int qknorm_version(void);
 
 #ifdef __cplusplus

@@ -39,7 +39,10 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) == {"qknorm_per_head", "qknorm_layerwise", "qknorm_status_string",
                           "qknorm_last_cuda_error", "qknorm_version", "qknorm_layerwise_partials",
                           "qknorm_layerwise_apply", "qknorm_layerwise_noalloc",
-                          "qknorm_wait_timeouts"}
+                          "qknorm_wait_timeouts", "qknorm_tp_comm_create",
+                          "qknorm_tp_comm_connect", "qknorm_tp_comm_create_local",
+                          "qknorm_tp_comm_destroy", "qknorm_tp_comm_errors",
+                          "qknorm_layerwise_tp_p2p"}
     for n in names:
         assert hasattr(lib, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", qbuild.LIB_PATH], capture_output=True,
@@ -49,7 +52,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.qknorm_version() == 104
+    assert lib.qknorm_version() == 105
     for code in (OK, NULL, SHAPE, ALIGN, NSHARDS, UNSUP, CUDA, EPS, -8):
         s = lib.qknorm_status_string(code).decode()
         assert s and s != "unknown status"

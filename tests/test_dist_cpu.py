@@ -180,3 +180,34 @@ def test_bench_gpus_flag_launches_that_many_ranks():
 def test_bench_gpus_flag_must_match_the_launcher():
     r = _bench(["--gpus", "2", "--dry-run"], {"WORLD_SIZE": "3", "RANK": "0"})
     assert r.returncode != 0 and "disagrees" in r.stderr
+
+
+def _handles_worker(rank, world, port, q):
+    """Every rank contributes a distinct 64-byte handle; every rank must get
+    all of them in rank order (what qknorm_tp_comm_connect expects)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+
+    import attention_qk_norm_b200 as qkn
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    mine = bytes([rank + 1]) * qkn._binding.IPC_HANDLE_BYTES
+    got = qkn.exchange_handles(mine)
+    q.put((rank, [h[0] for h in got], all(len(h) == 64 for h in got)))
+    dist.destroy_process_group()
+
+
+def test_ipc_handles_gathered_in_rank_order_gloo():
+    world = 4
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_handles_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == [(r, [1, 2, 3, 4], True) for r in range(world)]
