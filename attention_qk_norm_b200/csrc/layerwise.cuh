@@ -200,6 +200,12 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     constexpr int kEPT = VPT * kVec;  // elements per thread
     constexpr bool kOverlap = kSched == kSchedOverlap;
     constexpr bool kDirect = kSched == kSchedDirect;
+    // Every schedule sums squares in f32x2 pairs (sumsq_acc), so a head's
+    // partial is the same bits in every mode and schedule; the overlap
+    // schedule also forms its products on pairs, while the others, whose
+    // register caps leave no room for pair alignment, multiply in scalars
+    // (the same bits either way).
+    constexpr bool kPacked = kOverlap;
     constexpr int NST = kDirect ? 0 : kLayerwiseStages;  // stages of the ring
     constexpr bool kExchange = kCluster && kMode != kApply;
     // Vector loops unroll fully when gamma sits in registers (indexed by v);
@@ -318,6 +324,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
             if (Hk > 0) rk = rsqrtf(__ldg(aux + 2 * t + 1) * inv_len_k + eps);
         } else {
             float s = 0.f;
+            uint64_t acc = f2_pack(0.f, 0.f);
 #pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float f[kVec];
@@ -325,13 +332,18 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                     S::unpack(xr[v], f);
                 else
                     S::unpack(active ? sp[v * kLPH] : zero_vec<V>(), f);
+                sumsq_acc(acc, f);
+                if constexpr (kPacked) {
+                    float t[kVec];
+                    mul_elems(t, f, g + v * kVec);
 #pragma unroll
-                for (int e = 0; e < kVec; ++e) s = fmaf(f[e], f[e], s);
-                if constexpr (kOverlap) {
+                    for (int e = 0; e < kVec; ++e) xg[v * kVec + e] = t[e];
+                } else if constexpr (kOverlap) {
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) xg[v * kVec + e] = f[e] * g[v * kVec + e];
                 }
             }
+            s = sumsq_total(acc);
             s = group_sum<kLPH>(s);
             // Partials alternate between two buffers.  The next write into
             // this token's buffer is for the token after next; every block
@@ -440,7 +452,9 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #pragma unroll kUnroll
             for (int v = 0; v < VPT; ++v) {
                 float o[kVec];
-                if constexpr (kOverlap) {
+                if constexpr (kPacked) {
+                    mul_scalar(o, xg + v * kVec, rinv);
+                } else if constexpr (kOverlap) {
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) o[e] = xg[v * kVec + e] * rinv;
                 } else {
@@ -480,8 +494,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 // elements (and as many gamma values) per token.  The caps fit without
 // spilling and leave room for more resident blocks than the compiler's own
 // choice (up to 64); measured on B200 they are the fastest for every storage
-// type and head_dim.  The overlap and direct schedules also keep the thread's
-// x * gamma products, or its raw vectors, in registers: 48, 64 or 96.
+// type and head_dim.  FP8 threads with 32 elements (two 16-element vectors)
+// need 64 to decode a vector without spilling.  The overlap and direct
+// schedules also keep the thread's x * gamma products, or its raw vectors,
+// in registers: 48, 64 or 96.
 #ifndef QKN_LW_REGS8
 #define QKN_LW_REGS8 40
 #endif
@@ -500,11 +516,16 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
 #ifndef QKN_LW_OVERLAP_REGS32
 #define QKN_LW_OVERLAP_REGS32 96
 #endif
-__host__ __device__ constexpr int layerwise_regs(int ept, bool wide)
+#ifndef QKN_LW_REGS32_FP8
+#define QKN_LW_REGS32_FP8 64
+#endif
+__host__ __device__ constexpr int layerwise_regs(int ept, bool wide, int kvec)
 {
     return wide ? (ept <= 8 ? QKN_LW_OVERLAP_REGS8
                                : (ept <= 16 ? QKN_LW_OVERLAP_REGS16 : QKN_LW_OVERLAP_REGS32))
-                   : (ept <= 8 ? QKN_LW_REGS8 : (ept <= 16 ? QKN_LW_REGS16 : QKN_LW_REGS32));
+                   : (ept <= 8 ? QKN_LW_REGS8
+                               : (ept <= 16 ? QKN_LW_REGS16
+                                            : (kvec == 16 ? QKN_LW_REGS32_FP8 : QKN_LW_REGS32)));
 }
 
 // Gamma in registers (at most 32 elements per thread), with schedule kSched
@@ -513,7 +534,8 @@ __host__ __device__ constexpr int layerwise_regs(int ept, bool wide)
 // weight multiplication with the exchange), so after the combine only the
 // multiplication by the inverse RMS remains.
 template <typename TS, int D, int VPT, bool kCluster, int kMode, int kSched>
-__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kSched != kSchedRing)))
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, kSched != kSchedRing,
+                                             Storage<TS>::kVec)))
 qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                      const float *__restrict__ gamma_q, const float *__restrict__ gamma_k,
                      float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
@@ -538,7 +560,7 @@ struct TPRankPtrs {
 // blocks of the launch must be resident together (a cooperative launch),
 // since blocks of one token on different ranks wait for one another.
 template <typename TS, int D, int VPT>
-__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, true)))
+__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, true, Storage<TS>::kVec)))
 qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, int Hk,
                         float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
                         SumPlan plan_k, P2PArgs p2p)

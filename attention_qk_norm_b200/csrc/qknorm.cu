@@ -233,51 +233,10 @@ int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, 
                       gk, eps, (uint32_t)q_blocks);
 }
 
-template <typename TS, int D, bool kHasK>
-int launch_per_head_bulk(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride,
-                         const float *gq, const float *gk, float eps, cudaStream_t stream)
-{
-    using B = BulkShape<TS, D>;
-    auto kern = qkn_per_head_bulk_kernel<TS, D, kHasK>;
-    static KernelCache kc;
-    int dev = 0, per_sm = 0, rc;
-    DeviceInfo info;
-    if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
-    if (B::kSmemBytes > info.smem_optin) return QKN_ERR_UNSUPPORTED;
-    if ((rc = resident_blocks(kern, kc, dev, info, kBulkThreads, B::kSmemBytes, &per_sm)) != QKN_OK)
-        return rc;
-    if (per_sm < 1) return QKN_ERR_UNSUPPORTED;
-    const uint64_t rows = (uint64_t)T * (uint64_t)(Hq + Hk);
-    const uint64_t nchunks = (rows + B::kChunkRows - 1) / B::kChunkRows;
-    const uint64_t cap = (uint64_t)info.sms * per_sm;
-    const uint64_t grid = nchunks < cap ? nchunks : cap;
-    return launch_pdl(kern, (unsigned)grid, kBulkThreads, B::kSmemBytes, stream, 1u,
-                      static_cast<TS *>(qkv), row_stride, T, (uint32_t)(Hq + Hk), (uint32_t)Hq, gq,
-                      gk, eps, nchunks);
-}
-
-// Inputs of at least this many Q/K bytes take the bulk-staged kernel.
-#ifndef QKN_PH_BULK_MIN_BYTES
-#define QKN_PH_BULK_MIN_BYTES (1ll << 62)
-#endif
-#ifndef QKN_PH_BULK_MIN_BYTES_FP8
-#define QKN_PH_BULK_MIN_BYTES_FP8 (1ll << 62)
-#endif
-
 template <typename TS, int D>
 int launch_per_head(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                     const float *gk, float eps, cudaStream_t stream)
 {
-    const int64_t qk_bytes = T * (int64_t)(Hq + Hk) * D * (int64_t)sizeof(TS);
-    const int64_t bulk_min =
-        Storage<TS>::kVec == 16 ? (int64_t)QKN_PH_BULK_MIN_BYTES_FP8 : (int64_t)QKN_PH_BULK_MIN_BYTES;
-    if (qk_bytes >= bulk_min) {
-        if (Hq > 0 && Hk > 0)
-            return launch_per_head_bulk<TS, D, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
-                                                     stream);
-        return launch_per_head_bulk<TS, D, false>(qkv, T, Hq, Hk, row_stride, Hq > 0 ? gq : gk,
-                                                  nullptr, eps, stream);
-    }
     if (Hq > 0 && Hk > 0) {
         if constexpr (Storage<TS>::kVec == 16)  // FP8
             return launch_per_head_k<TS, D, false, true>(qkv, T, Hq, Hk, row_stride, gq, gk, eps,
@@ -499,12 +458,12 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
             // SMs shared, the ring with twice the VPT is 7% faster).
             if (kMode == kFused) sched = kSchedDirect;
         } else if (can_double &&
-                   T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false))) {
+                   T < kLayerwiseShortTokens * pipelines(layerwise_regs(ept, false, kVec))) {
             chosen *= 2;
             doubled = true;
         }
         if (!doubled && kMode == kFused && layerwise_overlap_type<TS>() && sched == kSchedRing &&
-            T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true)))
+            T >= kLayerwiseShortTokens * pipelines(layerwise_regs(ept, true, kVec)))
             sched = kSchedOverlap;
     }
     for (int vpt = 1; vpt <= kNV && chosen == 0; vpt *= 2)

@@ -189,7 +189,77 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// ---- mbarriers and bulk copies (the async proxy) --
+// ---- packed fp32 pairs --
+// sm_100 executes some fp32 operations on pairs of lanes held in a 64-bit
+// register pair (f32x2); each lane is rounded exactly as the scalar
+// instruction rounds it, so products come out bit-identical to scalar ones.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Sum of squares of a thread's elements.  With f32x2 the even- and the
+// odd-indexed elements accumulate in the two lanes of a pair (each in
+// element order), added at the end: a fixed order, the same in every kernel
+// and mode that sums a head.  acc starts at f2_pack(0, 0).
+template <int N>
+__device__ __forceinline__ void sumsq_acc(uint64_t &acc, const float (&f)[N])
+{
+    static_assert(N % 2 == 0, "pairs");
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        const uint64_t x = f2_pack(f[e], f[e + 1]);
+        acc = f2_fma(x, x, acc);
+    }
+}
+__device__ __forceinline__ float sumsq_total(uint64_t acc)
+{
+    float a, b;
+    f2_unpack(acc, a, b);
+    return a + b;
+}
+// o[e] = a[e] * b[e] for the N elements (b through a pointer into registers
+// or constants).
+template <int N>
+__device__ __forceinline__ void mul_elems(float (&o)[N], const float *a, const float *b)
+{
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        const uint64_t p = f2_mul(f2_pack(a[e], a[e + 1]), f2_pack(b[e], b[e + 1]));
+        f2_unpack(p, o[e], o[e + 1]);
+    }
+}
+// o[e] = a[e] * c for a scalar c.
+template <int N>
+__device__ __forceinline__ void mul_scalar(float (&o)[N], const float *a, float c)
+{
+    const uint64_t cc = f2_pack(c, c);
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        const uint64_t p = f2_mul(f2_pack(a[e], a[e + 1]), cc);
+        f2_unpack(p, o[e], o[e + 1]);
+    }
+}
+
+// ---- mbarriers and the global timer --
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -199,8 +269,7 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t arrivals)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(arrivals)
                  : "memory");
 }
-// Make initialised barriers visible to the async proxy and to the other
-// blocks of a cluster.
+// Make initialised barriers visible to the other blocks of a cluster.
 __device__ __forceinline__ void mbar_init_fence()
 {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -212,24 +281,6 @@ __device__ __forceinline__ void mbar_arm(uint64_t *bar, uint32_t bytes)
                  "r"(bytes)
                  : "memory");
 }
-// One plain arrival (release, CTA scope).
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Has the phase of parity `parity` completed?  (acquire, CTA scope)
-__device__ __forceinline__ bool mbar_try_wait_cta(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 __device__ __forceinline__ uint64_t global_ns()
 {
     uint64_t t;
@@ -237,39 +288,10 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// Every wait on a barrier gives up after this long (they complete in
-// microseconds when the hardware works); each give-up is counted in
-// g_wait_timeouts, which the host reads with qknorm_wait_timeouts.
+// Every bounded wait gives up after this long (they complete in microseconds
+// when the hardware works); each give-up is counted in g_wait_timeouts, which
+// the host reads with qknorm_wait_timeouts.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 __device__ unsigned int g_wait_timeouts;
-
-// Bounded wait on the phase of parity `parity` (CTA scope); false on time-out.
-__device__ __forceinline__ bool mbar_wait_cta_bounded(uint64_t *bar, uint32_t parity)
-{
-    if (mbar_try_wait_cta(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait_cta(bar, parity))
-        if (global_ns() - t0 > kWaitLimitNs) return false;
-    return true;
-}
-
-// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
-// from global to this block's shared memory, counted against `bar`'s
-// transaction bytes.  Evict-first in L2: every byte is read once.
-__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, uint32_t bytes,
-                                          uint64_t *bar, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
-        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-__device__ __forceinline__ uint64_t l2_evict_first_policy()
-{
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
 
 }  // namespace
