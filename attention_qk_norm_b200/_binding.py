@@ -308,6 +308,19 @@ def exchange_handles(handle: bytes, group=None):
     return out
 
 
+def _agree(ok: bool, group, what: str) -> None:
+    """All-reduce (min) a success flag over ``group``; raise on every rank if
+    any rank failed."""
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([1 if ok else 0], dtype=torch.int32, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN, group=group)
+    if int(t.item()) == 0:
+        raise RuntimeError(what)
+
+
 class TPComm:
     """Communicator of ``qknorm_layerwise_tp_p2p`` (see include/qknorm.h):
     this rank's receive buffer and the other ranks' buffers mapped through
@@ -343,16 +356,19 @@ class TPComm:
         lib = load_library()
         ptr = ctypes.c_void_p()
         handle = (ctypes.c_char * IPC_HANDLE_BYTES)()
-        _check("qknorm_tp_comm_create", lib.qknorm_tp_comm_create(
-            world, rank, int(max_tokens), float(timeout_s), ctypes.byref(ptr), handle))
+        rc = lib.qknorm_tp_comm_create(world, rank, int(max_tokens), float(timeout_s),
+                                       ctypes.byref(ptr), handle)
+        if world > 1:
+            # Every rank learns whether all created their buffer before any
+            # collective that a failed rank would not join.
+            _agree(rc == 0, group, "qknorm_tp_comm_create failed on some rank")
+        _check("qknorm_tp_comm_create", rc)
         comm = cls(ptr, world, rank, 1, group)
         handles = exchange_handles(bytes(handle), group)
         if world > 1:
             torch.cuda.synchronize()
-            dist.barrier(group)  # every rank's buffer exists before any opens it
-            joined = b"".join(handles)
-            _check("qknorm_tp_comm_connect", lib.qknorm_tp_comm_connect(ptr, joined))
-            dist.barrier(group)
+            rc = lib.qknorm_tp_comm_connect(ptr, b"".join(handles))
+            _agree(rc == 0, group, "qknorm_tp_comm_connect failed on some rank")
         return comm
 
     def errors(self) -> int:

@@ -8,7 +8,6 @@
 #include <cooperative_groups.h>
 
 #include "storage.cuh"
-#include "tp_exchange.h"
 
 namespace {
 
@@ -107,57 +106,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 //              over all ranks and len_q, len_k the full vector lengths.
 // The mean S/L is formed as S * inv_len with inv_len = 1/L rounded to fp32
 // once per launch.
-//   kP2P:      tensor-parallel layerwise QK-Norm in one launch per rank: this
-//              rank's two sums of squares are stored into every rank's
-//              receive buffer (peer stores, see tp_exchange.h), the world
-//              ranks' sums of the token are read back from this rank's own
-//              buffer and combined in a fixed tree, and the rank's columns
-//              are scaled with the full lengths; x * gamma is formed before
-//              the exchange (the overlap schedule).
-enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2, kP2P = 3 };
-
-// The exchange of a kP2P launch (tp_exchange.h).
-struct P2PArgs {
-    uint64_t *recv[qkn_tp::kMaxWorld];  // every rank's receive buffer, as this GPU addresses it
-    unsigned int *errors;               // the group's count of waits that gave up
-    uint32_t *abort_tag;                // tag of a call in which a wait gave up
-    int64_t max_tokens;
-    uint64_t timeout_ns;
-    int world;
-    int rank;                           // rank of grid row 0 (blockIdx.y adds to it)
-    uint32_t parity, tag;
-};
-
-// 64-bit relaxed accesses at system scope: a peer's stores over NVLink and
-// this GPU's polls of them.  Each is single-copy atomic (naturally aligned).
-__device__ __forceinline__ void st_relaxed_sys_u64(uint64_t *p, uint64_t v)
-{
-    asm volatile("st.relaxed.sys.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t ld_relaxed_sys_u64(const uint64_t *p)
-{
-    uint64_t v;
-    asm volatile("ld.relaxed.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Element i of a small pointer array held in kernel parameters, with a
-// compile-time index on every access (no copy of the array to local memory).
-template <typename P, int N>
-__device__ __forceinline__ P pick(const P (&a)[N], int i)
-{
-    P r = a[0];
-#pragma unroll
-    for (int j = 1; j < N; ++j)
-        if (j == i) r = a[j];
-    return r;
-}
+enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 
 // How a launch moves each token through its block.
 //   kSchedRing:    a two-stage cp.async ring in shared memory (the next token
@@ -189,7 +138,7 @@ __device__ __forceinline__ void
 layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, int Hk,
                  const float *__restrict__ gamma_q, const float *__restrict__ gamma_k, float eps,
                  float inv_len_q, float inv_len_k, SumPlan plan_q, SumPlan plan_k,
-                 float *__restrict__ aux, const P2PArgs *p2p = nullptr)
+                 float *__restrict__ aux)
 {
     using S = Storage<TS>;
     using V = typename S::Vec;
@@ -240,14 +189,6 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
 
     pdl_wait_then_release();
-    // kP2P: lane r of a warp stores to, and polls the slot of, rank r.
-    uint64_t *peer_buf = nullptr;
-    const uint64_t *own_buf = nullptr;
-    bool gave_up = false;
-    if constexpr (kMode == kP2P) {
-        peer_buf = pick(p2p->recv, lane);
-        own_buf = pick(p2p->recv, p2p->rank + (int)blockIdx.y);
-    }
     // This thread's head weights (the partials step has none).
     const float *gb = gamma_q;
     if (kMode != kPartials && active)
@@ -373,65 +314,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 if (active && l == 0) pp[h] = s;
                 __syncthreads();
             }
-            if constexpr (kMode == kP2P) {
-                const int world = p2p->world;
-                const int me = p2p->rank + (int)blockIdx.y;
-                if (threadIdx.x < 32) {  // warp 0 sends this rank's two sums to every rank
-                    const float sq = warp_sumsq(pp, plan_q, lane);
-                    const float sk = warp_sumsq(pp + Hq, plan_k, lane);
-                    if (lane < world) {
-                        uint64_t *dst = peer_buf + qkn_tp::slot_word(p2p->parity, t, me, 0,
-                                                                     p2p->max_tokens, world);
-                        st_relaxed_sys_u64(dst, qkn_tp::pack(sq, p2p->tag));
-                        st_relaxed_sys_u64(dst + 1, qkn_tp::pack(sk, p2p->tag));
-                    }
-                }
-                if (need_q || need_k) {  // the world ranks' sums, from this rank's buffer
-                    float vq = 0.f, vk = 0.f;
-                    bool ok = true;
-                    if (lane < world) {
-                        const uint64_t *src =
-                            own_buf + qkn_tp::slot_word(p2p->parity, t, lane, 0, p2p->max_tokens,
-                                                        world);
-                        uint64_t wq = ld_relaxed_sys_u64(src), wk = ld_relaxed_sys_u64(src + 1);
-                        if (!gave_up &&
-                            !(qkn_tp::arrived(wq, p2p->tag) && qkn_tp::arrived(wk, p2p->tag))) {
-                            const uint64_t t0 = global_ns();
-                            for (;;) {
-                                wq = ld_relaxed_sys_u64(src);
-                                wk = ld_relaxed_sys_u64(src + 1);
-                                if (qkn_tp::arrived(wq, p2p->tag) && qkn_tp::arrived(wk, p2p->tag))
-                                    break;
-                                if (global_ns() - t0 > p2p->timeout_ns ||
-                                    ld_relaxed_gpu_u32(p2p->abort_tag) == p2p->tag) {
-                                    ok = false;
-                                    break;
-                                }
-                            }
-                        }
-                        vq = qkn_tp::value_of(wq);
-                        vk = qkn_tp::value_of(wk);
-                    }
-                    if (__any_sync(0xffffffffu, !ok) && !gave_up) {
-                        // Count it, tell the other blocks, and wait no more in
-                        // this launch (its outputs are wrong from here on).
-                        gave_up = true;
-                        if (lane == 0) {
-                            atomicAdd(p2p->errors, 1u);
-                            atomicAdd(&g_wait_timeouts, 1u);
-                            atomicExch(p2p->abort_tag, p2p->tag);
-                        }
-                    }
-                    for (int d = 1; d < world; d <<= 1) {  // fixed rank tree, tp_exchange.h
-                        vq += __shfl_xor_sync(0xffffffffu, vq, d);
-                        vk += __shfl_xor_sync(0xffffffffu, vk, d);
-                    }
-                    vq = __shfl_sync(0xffffffffu, vq, 0);
-                    vk = __shfl_sync(0xffffffffu, vk, 0);
-                    if (need_q) rq = rsqrtf(vq * inv_len_q + eps);
-                    if (need_k) rk = rsqrtf(vk * inv_len_k + eps);
-                }
-            } else if constexpr (kMode == kPartials) {
+            if constexpr (kMode == kPartials) {
                 // One warp of the cluster's first block writes this rank's sums.
                 if (threadIdx.x < 32 && crank == 0) {
                     const float sq = warp_sumsq(pp, plan_q, lane);
@@ -544,31 +427,6 @@ qkn_layerwise_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq
     layerwise_tokens<TS, D, VPT, true, kCluster, kMode, kSched>(
         qkv, row_stride, T, Hq, Hk, gamma_q, gamma_k, eps, inv_len_q, inv_len_k, plan_q, plan_k,
         aux);
-}
-
-// Pointers of the ranks one kP2P launch serves: one (a rank on its own GPU)
-// or every rank of a group emulated on one GPU (grid row y serves rank
-// p2p.rank + y).
-struct TPRankPtrs {
-    void *qkv[qkn_tp::kMaxWorld];
-    const float *gamma_q[qkn_tp::kMaxWorld];
-    const float *gamma_k[qkn_tp::kMaxWorld];
-};
-
-// Tensor-parallel layerwise QK-Norm with the exchange inside the kernel
-// (kP2P, overlap schedule, one block per token, gamma in registers).  All
-// blocks of the launch must be resident together (a cooperative launch),
-// since blocks of one token on different ranks wait for one another.
-template <typename TS, int D, int VPT>
-__global__ void __maxnreg__((layerwise_regs(VPT * Storage<TS>::kVec, true, Storage<TS>::kVec)))
-qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, int Hk,
-                        float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
-                        SumPlan plan_k, P2PArgs p2p)
-{
-    const int y = (int)blockIdx.y;
-    layerwise_tokens<TS, D, VPT, true, false, kP2P, kSchedOverlap>(
-        static_cast<TS *>(pick(ptrs.qkv, y)), row_stride, T, Hq, Hk, pick(ptrs.gamma_q, y),
-        pick(ptrs.gamma_k, y), eps, inv_len_q, inv_len_k, plan_q, plan_k, nullptr, &p2p);
 }
 
 // Gamma read through L1 (tokens too wide for registers; one block per token,

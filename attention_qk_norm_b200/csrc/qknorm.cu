@@ -52,6 +52,7 @@
 #include "layerwise.cuh"
 #include "per_head.cuh"
 #include "storage.cuh"
+#include "tp_kernel.cuh"
 
 namespace {
 
@@ -513,9 +514,9 @@ int dispatch(int dtype, int D, Args... args)
 }
 
 // ---------------------------------------- tensor-parallel exchange, P2P --
-// Launch shape of the in-kernel exchange: one block per token (no cluster),
-// gamma in registers, the fewest vectors per thread (at least 2) within 576
-// threads.
+// Launch shape of the in-kernel exchange (tp_kernel.cuh): one block per
+// token (no cluster), gamma in registers, the fewest vectors per thread (at
+// least 2) within 576 threads.
 template <typename TS, int D, int VPT>
 int launch_tp_vpt(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
                   int64_t row_stride, float eps, float inv_len_q, float inv_len_k, SumPlan plan_q,
@@ -525,7 +526,7 @@ int launch_tp_vpt(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
     static KernelCache kc;
     const int heads = Hq + Hk;
     const size_t span = (size_t)heads * D * sizeof(TS);
-    const size_t smem = kLayerwiseStages * span + (size_t)2 * heads * sizeof(float);
+    const size_t smem = kTPStages * span + (size_t)2 * heads * sizeof(float);
     int dev = 0, per_sm = 0, rc;
     DeviceInfo info;
     if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;

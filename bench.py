@@ -404,6 +404,13 @@ def run_tp(device, l2, world, rank, T_list=(1, 16, 256, 4096, 8192)):
     gk_full = 1.0 + 0.1 * torch.randn(G["Hk"] * D, generator=gen, device=device)
     gq = gq_full[rank * hq * D:(rank + 1) * hq * D].contiguous()
     gk = gk_full[rank * hk * D:(rank + 1) * hk * D].contiguous()
+    # The in-kernel exchange over the same group (peer stores through CUDA
+    # IPC); any failure is reported, not raised, so the line still prints.
+    comm, p2p_error = None, None
+    try:
+        comm = qkn.TPComm.from_group(max_tokens=max(T_list), timeout_s=10.0)
+    except Exception as ex:  # every rank raises together (TPComm.from_group)
+        p2p_error = str(ex)[:200]
     points = []
     for T in T_list:
         d = synth.make_case_torch(T, hq, hk, D, device=device, layerwise=True,
@@ -416,18 +423,104 @@ def run_tp(device, l2, world, rank, T_list=(1, 16, 256, 4096, 8192)):
         ag = time_eager_us(lambda b: qkn.qknorm_layerwise_tp_allgather(b, hq, hk, D, gq_full,
                                                                        gk_full, eps),
                            bufs, world)
-        points.append({"T": T, "scalar_allreduce_us": round(ar, 3),
-                       "allgather_us": round(ag, 3),
-                       "allreduce_vs_allgather": round(ar / ag, 4)})
+        pt = {"T": T, "scalar_allreduce_us": round(ar, 3), "allgather_us": round(ag, 3),
+              "allreduce_vs_allgather": round(ar / ag, 4)}
+        if comm is not None:
+            p2p = time_eager_us(
+                lambda b: qkn.qknorm_layerwise_tp_p2p(comm, b, hq, hk, D, gq, gk, eps), bufs,
+                world)
+            pt["in_kernel_p2p_us"] = round(p2p, 3)
+            pt["p2p_vs_allgather"] = round(p2p / ag, 4)
+        points.append(pt)
         del bufs, d
         torch.cuda.empty_cache()
-    return {"world": world, "heads_per_rank": {"q": hq, "kv": hk}, "head_dim": D,
-            "dtype": G["dtype"],
-            "workload": "layerwise QK-Norm of 32 query / 8 key heads x 128 split by head over "
-                        "%d rank(s), one layer call per step" % world,
-            "timing": "eager calls (they hold NCCL collectives), CUDA events, mean of 50, "
-                      "max over ranks",
+    out = {"world": world, "heads_per_rank": {"q": hq, "kv": hk}, "head_dim": D,
+           "dtype": G["dtype"],
+           "workload": "layerwise QK-Norm of 32 query / 8 key heads x 128 split by head over "
+                       "%d rank(s), one layer call per step" % world,
+           "timing": "eager calls through the Python binding (the exchanges hold NCCL "
+                     "collectives), CUDA events, mean of 50, max over ranks",
+           "points": points}
+    if comm is not None:
+        torch.cuda.synchronize()
+        out["in_kernel_p2p_waits_given_up"] = int(max_over_ranks(float(comm.errors()), world))
+        comm.close()
+    else:
+        out["in_kernel_p2p_error"] = p2p_error
+    out["emulated_group"] = run_tp_emulated(device, l2, world)
+    return out
+
+
+def run_tp_emulated(device, l2, world, ranks=8, T_list=(1, 16, 256, 4096, 8192)):
+    """An 8-rank group emulated on this GPU: every rank's buffer and receive
+    buffer here, all ranks served by one cooperative launch of the in-kernel
+    exchange, against the fused single-GPU kernel with nshards = 8 over the
+    whole vectors (no exchange at all).  Graphs of 50 launches, CUDA events,
+    max over ranks."""
+    import torch
+    import attention_qk_norm_b200 as qkn
+    from attention_qk_norm_b200 import synth
+
+    G = TP_GLOBAL
+    hq, hk, D, eps = G["Hq"] // ranks, G["Hk"] // ranks, G["D"], G["eps"]
+    comm = qkn.TPComm.local(ranks, max_tokens=max(T_list), timeout_s=10.0)
+    points = []
+    for T in T_list:
+        d = synth.make_case_torch(T, G["Hq"], G["Hk"], D, device=device, layerwise=True,
+                                  seed=3100 + T)
+        W = (hq + 2 * hk) * D
+        one = d["qkv"].numel() * d["qkv"].element_size()
+        n = max(2, min(32, math.ceil(4 * l2 / max(1, one))))
+        full = [d["qkv"].clone() for _ in range(n)]
+        parts = [[d["qkv"][:, :W].clone() for _ in range(ranks)] for _ in range(n)]
+        gqs = [d["gamma_q"][r * hq * D:(r + 1) * hq * D].contiguous() for r in range(ranks)]
+        gks = [d["gamma_k"][r * hk * D:(r + 1) * hk * D].contiguous() for r in range(ranks)]
+        p2p = time_graph_fn_us(
+            lambda i: qkn.qknorm_layerwise_tp_p2p(comm, parts[i], hq, hk, D, gqs, gks, eps), n)
+        fused = time_graph_fn_us(
+            lambda i: qkn.qknorm_layerwise(full[i], G["Hq"], G["Hk"], D, d["gamma_q"],
+                                           d["gamma_k"], eps, nshards=ranks), n)
+        points.append({"T": T, "in_kernel_p2p_group_us": round(max_over_ranks(p2p, world), 3),
+                       "fused_nshards8_us": round(max_over_ranks(fused, world), 3)})
+        del full, parts, d
+        torch.cuda.empty_cache()
+    torch.cuda.synchronize()
+    errors = comm.errors()
+    comm.close()
+    return {"ranks": ranks, "heads_per_rank": {"q": hq, "kv": hk}, "waits_given_up": errors,
             "points": points}
+
+
+def time_graph_fn_us(fn, nbufs, steps=50, reps=5):
+    """Median µs per call of ``fn(i)`` (i rotating over ``nbufs`` buffers)
+    replayed from a CUDA graph of ``steps`` calls."""
+    import torch
+
+    i = [0]
+
+    def launch():
+        fn(i[0] % nbufs)
+        i[0] += 1
+
+    for _ in range(3):
+        launch()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps):
+            launch()
+    g.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for _ in range(reps):
+        s.record()
+        g.replay()
+        e.record()
+        e.synchronize()
+        out.append(s.elapsed_time(e) * 1e3 / steps)
+    del g
+    return statistics.median(out)
 
 
 def e2e(w, device, steps, lanes=2):
@@ -521,14 +614,34 @@ def run_ours(args):
     hbm_peak, peak_kind = peaks()
     w = dict(HEADLINE)
     wl = Workload(w, device, l2)
-    full, rem = divmod(args.steps, GRAPH_STEPS)
-    g_full = wl.graph(GRAPH_STEPS) if full else None
-    g_rem = wl.graph(rem) if rem else None
+    # The K timed steps as graphs of up to GRAPH_STEPS launches: the first
+    # graph opens with the start event and the last one closes with the end
+    # event (event nodes inside the graphs), so the timed region is the K
+    # launches on the device, without the host's graph-launch latency.
+    s = torch.cuda.Event(enable_timing=True, external=True)
+    e = torch.cuda.Event(enable_timing=True, external=True)
+    sizes = [GRAPH_STEPS] * (args.steps // GRAPH_STEPS)
+    if args.steps % GRAPH_STEPS:
+        sizes.append(args.steps % GRAPH_STEPS)
+    timed = []  # (graph, replays)
+    for j, n in enumerate(sizes):
+        first, last = j == 0, j == len(sizes) - 1
+        if not first and not last and timed and timed[-1][2]:
+            timed[-1][1] += 1  # another replay of the plain middle graph
+            continue
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if first:
+                s.record()
+            for _ in range(n):
+                wl.launch()
+            if last:
+                e.record()
+        timed.append([g, 1, not first and not last])
     # Replay every graph once: a graph's first replay uploads it to the
     # device, which must not land inside the timed region.
-    for g in (g_full, g_rem):
-        if g is not None:
-            g.replay()
+    for g, _, _ in timed:
+        g.replay()
     torch.cuda.synchronize()
 
     # The clock sampler starts first; while it comes up the GPU replays a
@@ -549,19 +662,15 @@ def run_ours(args):
         wl.launch()
     barrier(world)
     torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(full):
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    e.record()
+    for g, replays, _ in timed:
+        for _ in range(replays):
+            g.replay()
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop() if rank == 0 else None
     ms_local = s.elapsed_time(e)
     ms = max_over_ranks(ms_local, world)
-    del g_full, g_rem
+    del timed
 
     steps = args.steps
     tokens = w["T"] * steps * world
