@@ -794,6 +794,10 @@ PROFILE_CASES = {
                            seed=1004),
     "layerwise_fp8": dict(kind="layerwise", T=32768, Hq=32, Hk=8, D=128, dtype="fp8_e4m3",
                           eps=1e-6, nshards=8, seed=1006),
+    # The in-kernel tensor-parallel exchange, an 8-rank group emulated on one
+    # GPU (one cooperative launch serves all ranks).
+    "tp_group": dict(kind="tp_group", T=4096, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
+                     nshards=8, seed=1007),
     # 128 heads of 256: too wide for one block, so 2-block clusters exchange
     # head partials through distributed shared memory.
     "layerwise_cluster": dict(kind="layerwise", T=4096, Hq=112, Hk=16, D=256, dtype="bf16",
@@ -816,6 +820,28 @@ def run_profile(args):
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(device)
     props = torch.cuda.get_device_properties(device)
+    if w["kind"] == "tp_group":
+        import attention_qk_norm_b200 as qkn
+        from attention_qk_norm_b200 import synth
+
+        n = w["nshards"]
+        hq, hk, D = w["Hq"] // n, w["Hk"] // n, w["D"]
+        d = synth.make_case_torch(w["T"], w["Hq"], w["Hk"], D, device=device, layerwise=True,
+                                  seed=w["seed"])
+        W = (hq + 2 * hk) * D
+        reps = max(2, math.ceil(4 * props.L2_cache_size / (d["qkv"].numel() * 2)))
+        parts = [[d["qkv"][:, :W].clone() for _ in range(n)] for _ in range(reps)]
+        gqs = [d["gamma_q"][r * hq * D:(r + 1) * hq * D].contiguous() for r in range(n)]
+        gks = [d["gamma_k"][r * hk * D:(r + 1) * hk * D].contiguous() for r in range(n)]
+        comm = qkn.TPComm.local(n, max_tokens=w["T"])
+        for i in range(args.warmup + args.steps):
+            qkn.qknorm_layerwise_tp_p2p(comm, parts[i % reps], hq, hk, D, gqs, gks, w["eps"])
+        torch.cuda.synchronize()
+        comm.close()
+        print(json.dumps({"profile": args.profile, "T": w["T"], "ranks": n,
+                          "launches": args.warmup + args.steps,
+                          "bytes_per_launch": workload_bytes(dict(w, kind="layerwise"))}))
+        return
     wl = Workload(w, device, l2_bytes=int(getattr(props, "L2_cache_size", 126 << 20)),
                   max_bytes=4 << 30)
     for _ in range(args.warmup + args.steps):
