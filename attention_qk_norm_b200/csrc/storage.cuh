@@ -90,37 +90,53 @@ struct Storage<__half> {
 // FP8 E4M3 (bias 7, no infinities, largest finite 448): 16 per 16-byte
 // vector.  Decoded exactly through fp16; encoded round-to-nearest-even,
 // saturating to +-448.  The lower byte of each pair is the earlier element.
+// Each 32-bit word is split into, and rebuilt from, its two 16-bit halves by
+// register moves, which the conversions take and produce directly, so no
+// shift or mask instruction is spent on a pair.
+__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float &f0, float &f1, float &f2, float &f3)
+{
+    asm("{\n\t.reg .b16 lo, hi, a0, a1, a2, a3;\n\t.reg .b32 h0, h1;\n\t"
+        "mov.b32 {lo, hi}, %4;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h0, lo;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h1, hi;\n\t"
+        "mov.b32 {a0, a1}, h0;\n\t"
+        "mov.b32 {a2, a3}, h1;\n\t"
+        "cvt.f32.f16 %0, a0;\n\t"
+        "cvt.f32.f16 %1, a1;\n\t"
+        "cvt.f32.f16 %2, a2;\n\t"
+        "cvt.f32.f16 %3, a3;\n\t}"
+        : "=f"(f0), "=f"(f1), "=f"(f2), "=f"(f3)
+        : "r"(w));
+}
+__device__ __forceinline__ uint32_t f32_to_e4m3x4(float f0, float f1, float f2, float f3)
+{
+    uint32_t w;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"  // upper byte f1, lower byte f0
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(w)
+        : "f"(f0), "f"(f1), "f"(f2), "f"(f3));
+    return w;
+}
+
 template <>
 struct Storage<__nv_fp8_e4m3> {
     using Vec = uint4;
     static constexpr int kVec = 16;
     __device__ __forceinline__ static void unpack(const uint4 &v, float (&f)[16])
     {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(
-                    (__nv_fp8x2_storage_t)((w[i] >> (16 * j)) & 0xffffu), __NV_E4M3);
-                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&r));
-                f[4 * i + 2 * j] = p.x;
-                f[4 * i + 2 * j + 1] = p.y;
-            }
-        }
+        e4m3x4_to_f32(v.x, f[0], f[1], f[2], f[3]);
+        e4m3x4_to_f32(v.y, f[4], f[5], f[6], f[7]);
+        e4m3x4_to_f32(v.z, f[8], f[9], f[10], f[11]);
+        e4m3x4_to_f32(v.w, f[12], f[13], f[14], f[15]);
     }
     __device__ __forceinline__ static uint4 pack(const float (&f)[16])
     {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i], f[4 * i + 1]),
-                                                         __NV_SATFINITE, __NV_E4M3);
-            const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f[4 * i + 2], f[4 * i + 3]),
-                                                         __NV_SATFINITE, __NV_E4M3);
-            w[i] = lo | (hi << 16);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
+        return make_uint4(f32_to_e4m3x4(f[0], f[1], f[2], f[3]),
+                          f32_to_e4m3x4(f[4], f[5], f[6], f[7]),
+                          f32_to_e4m3x4(f[8], f[9], f[10], f[11]),
+                          f32_to_e4m3x4(f[12], f[13], f[14], f[15]));
     }
 };
 
