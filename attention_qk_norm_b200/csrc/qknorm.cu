@@ -648,7 +648,6 @@ int noalloc_scratch(float **out)
 struct qkn_tp_comm {
     int world = 0, rank = 0, nlocal = 0, device = -1;
     int64_t max_tokens = 0;
-    uint64_t calls = 0;
     uint64_t timeout_ns = 0;
     bool connected = false;
     uint64_t *own[qkn_tp::kMaxWorld] = {};   // buffers this communicator allocated
@@ -656,6 +655,8 @@ struct qkn_tp_comm {
     bool opened[qkn_tp::kMaxWorld] = {};     // recv[r] is an IPC mapping to close
     unsigned int *errors = nullptr;          // device counter of waits that gave up
     uint32_t *abort_tag = nullptr;
+    uint32_t *seq = nullptr;                 // device: calls made so far (advanced by each launch)
+    uint32_t *done = nullptr;                // device: blocks of the running launch that finished
 };
 
 namespace {
@@ -679,7 +680,9 @@ int tp_alloc(qkn_tp_comm *c, int n)
     }
     unsigned char *tail = reinterpret_cast<unsigned char *>(c->own[0]) + bytes;
     c->errors = reinterpret_cast<unsigned int *>(tail);
-    c->abort_tag = reinterpret_cast<uint32_t *>(tail + 128);
+    c->abort_tag = reinterpret_cast<uint32_t *>(tail + 64);
+    c->seq = reinterpret_cast<uint32_t *>(tail + 128);
+    c->done = reinterpret_cast<uint32_t *>(tail + 192);
     return QKN_OK;
 }
 
@@ -885,7 +888,6 @@ int qknorm_layerwise_tp_p2p(qkn_tp_comm *comm, void *const *qkv, int dtype, int6
     if (T > comm->max_tokens) return QKN_ERR_TOO_LARGE;
     if (done) return QKN_OK;
     if (!comm->connected) return QKN_ERR_UNSUPPORTED;
-    if (comm->calls >= qkn_tp::kMaxCalls) return QKN_ERR_TOO_LARGE;
     int dev = -1;
     const cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -900,18 +902,16 @@ int qknorm_layerwise_tp_p2p(qkn_tp_comm *comm, void *const *qkv, int dtype, int6
     for (int r = 0; r < comm->world; ++r) a.recv[r] = comm->recv[r];
     a.errors = comm->errors;
     a.abort_tag = comm->abort_tag;
+    a.seq = comm->seq;
+    a.done = comm->done;
     a.max_tokens = comm->max_tokens;
     a.timeout_ns = comm->timeout_ns;
     a.world = comm->world;
     a.rank = comm->rank;
-    a.parity = qkn_tp::call_parity(comm->calls);
-    a.tag = qkn_tp::call_tag(comm->calls);
     const float len_q = (float)((int64_t)Hq * D * comm->world);
     const float len_k = (float)((int64_t)Hk * D * comm->world);
-    const int rc = dispatch<LayerwiseTP>(dtype, D, ptrs, comm->nlocal, T, Hq, Hk, row_stride, eps,
-                                         len_q, len_k, a, static_cast<cudaStream_t>(stream));
-    if (rc == QKN_OK) ++comm->calls;
-    return rc;
+    return dispatch<LayerwiseTP>(dtype, D, ptrs, comm->nlocal, T, Hq, Hk, row_stride, eps, len_q,
+                                 len_k, a, static_cast<cudaStream_t>(stream));
 }
 
 const char *qknorm_status_string(int status)

@@ -62,13 +62,13 @@ QKN_TP_HD uint64_t slot_word(uint32_t parity, int64_t t, int src, int which, int
            (uint64_t)which;
 }
 
-// Parity and tag of the call with (0-based) sequence number `call`: the
-// parity alternates, the tag grows by one per call of the same parity and
-// is never 0 (the value of a slot never written).
-QKN_TP_HD uint32_t call_parity(uint64_t call) { return (uint32_t)(call & 1u); }
-QKN_TP_HD uint32_t call_tag(uint64_t call) { return (uint32_t)(call >> 1) + 1u; }
-// Calls beyond this would reuse a tag; a communicator refuses them.
-constexpr uint64_t kMaxCalls = 2ull * 0xFFFFFFFEull;
+// Parity and tag of the call with (0-based) sequence number `call`, a 32-bit
+// count of the communicator's calls: the parity alternates, the tag grows by
+// one per call of the same parity and is never 0 (the value of a slot never
+// written).  After 2^32 calls the count wraps and tags repeat; a slot could
+// then be taken for fresh only if no call in those 2^32 wrote it.
+QKN_TP_HD uint32_t call_parity(uint32_t call) { return call & 1u; }
+QKN_TP_HD uint32_t call_tag(uint32_t call) { return (call >> 1) + 1u; }
 
 QKN_TP_HD uint32_t f32_bits(float v)
 {

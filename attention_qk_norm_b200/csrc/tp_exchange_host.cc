@@ -37,7 +37,7 @@ extern "C" int qkn_tp_host_rank_call(uint64_t *const *recv, int world, int rank,
     if (world < 1 || world > qkn_tp::kMaxWorld || rank < 0 || rank >= world || blocks < 1 ||
         T > max_tokens)
         return -1;
-    const uint32_t parity = qkn_tp::call_parity(call), tag = qkn_tp::call_tag(call);
+    const uint32_t parity = qkn_tp::call_parity((uint32_t)call), tag = qkn_tp::call_tag((uint32_t)call);
     std::atomic<bool> abort_call{false};
     std::atomic<int> gave_up_total{0};
     auto block = [&](int b) {

@@ -16,6 +16,11 @@
 // with work (SwiftQK review, key_machinery), taken one token further than
 // overlapping only the weight multiplication.
 //
+// Calls: the sequence number of the call (which picks the buffer half and
+// the tag) is read from device memory when the launch starts and advanced by
+// the launch's last block, so consecutive launches, replayed graphs
+// included, always carry consecutive sequence numbers.
+//
 // Deadlock freedom: a block's poll for t_{i-1} waits for the blocks of the
 // same index on the other ranks to have sent t_{i-1}, which each does in its
 // iteration i-1 before it polls anything of iteration i-1 itself; so by
@@ -32,16 +37,19 @@
 
 namespace {
 
-// The exchange of one launch.
+// The exchange of one launch.  The call's sequence number lives in device
+// memory: every block reads it when the launch starts, and the last block to
+// finish advances it, so launches replayed from a CUDA graph get new tags.
 struct P2PArgs {
     uint64_t *recv[qkn_tp::kMaxWorld];  // every rank's receive buffer, as this GPU addresses it
     unsigned int *errors;               // the group's count of waits that gave up
     uint32_t *abort_tag;                // tag of a call in which a wait gave up
+    uint32_t *seq;                      // calls made on this GPU's communicator so far
+    uint32_t *done;                     // blocks of the current launch that have finished
     int64_t max_tokens;
     uint64_t timeout_ns;
     int world;
     int rank;                           // rank of grid row 0 (blockIdx.y adds to it)
-    uint32_t parity, tag;
 };
 
 // Pointers of the ranks one launch serves: one (a rank on its own GPU) or
@@ -125,6 +133,10 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
     const int64_t first = blockIdx.x, stride = gridDim.x;
 
     pdl_wait_then_release();
+    // This call's buffer half and tag (tp_exchange.h), from the sequence
+    // number that the previous launch left behind.
+    const uint32_t call = ld_relaxed_gpu_u32(p2p.seq);
+    const uint32_t parity = qkn_tp::call_parity(call), tag = qkn_tp::call_tag(call);
     // Lane r of a warp stores to, and polls the slot of, rank r.
     uint64_t *const peer_buf = pick(p2p.recv, lane);
     const uint64_t *const own_buf = pick(p2p.recv, me);
@@ -175,16 +187,16 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
             bool ok = true;
             if (lane < world) {
                 const uint64_t *src =
-                    own_buf + qkn_tp::slot_word(p2p.parity, t, lane, 0, p2p.max_tokens, world);
+                    own_buf + qkn_tp::slot_word(parity, t, lane, 0, p2p.max_tokens, world);
                 uint64_t wq = ld_relaxed_sys_u64(src), wk = ld_relaxed_sys_u64(src + 1);
-                if (!gave_up && !(qkn_tp::arrived(wq, p2p.tag) && qkn_tp::arrived(wk, p2p.tag))) {
+                if (!gave_up && !(qkn_tp::arrived(wq, tag) && qkn_tp::arrived(wk, tag))) {
                     const uint64_t t0 = global_ns();
                     for (;;) {
                         wq = ld_relaxed_sys_u64(src);
                         wk = ld_relaxed_sys_u64(src + 1);
-                        if (qkn_tp::arrived(wq, p2p.tag) && qkn_tp::arrived(wk, p2p.tag)) break;
+                        if (qkn_tp::arrived(wq, tag) && qkn_tp::arrived(wk, tag)) break;
                         if (global_ns() - t0 > p2p.timeout_ns ||
-                            ld_relaxed_gpu_u32(p2p.abort_tag) == p2p.tag) {
+                            ld_relaxed_gpu_u32(p2p.abort_tag) == tag) {
                             ok = false;
                             break;
                         }
@@ -200,7 +212,7 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
                 if (lane == 0) {
                     atomicAdd(p2p.errors, 1u);
                     atomicAdd(&g_wait_timeouts, 1u);
-                    atomicExch(p2p.abort_tag, p2p.tag);
+                    atomicExch(p2p.abort_tag, tag);
                 }
             }
             for (int d = 1; d < world; d <<= 1) {  // the fixed rank tree (tp_exchange.h)
@@ -253,9 +265,9 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
             const float sk = warp_sumsq(pp + Hq, plan_k, lane);
             if (lane < world) {
                 uint64_t *dst =
-                    peer_buf + qkn_tp::slot_word(p2p.parity, t, me, 0, p2p.max_tokens, world);
-                st_relaxed_sys_u64(dst, qkn_tp::pack(sq, p2p.tag));
-                st_relaxed_sys_u64(dst + 1, qkn_tp::pack(sk, p2p.tag));
+                    peer_buf + qkn_tp::slot_word(parity, t, me, 0, p2p.max_tokens, world);
+                st_relaxed_sys_u64(dst, qkn_tp::pack(sq, tag));
+                st_relaxed_sys_u64(dst + 1, qkn_tp::pack(sk, tag));
             }
         }
         if (tprev >= 0) finish(tprev, gprev, sp_prev);
@@ -269,6 +281,16 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
     }
     if (tprev >= 0) finish(tprev, gprev, sp_prev);
     cp_async_wait<0>();
+    // The last block of the launch to finish advances the sequence number
+    // (every block has read it by then: it read it before its first token).
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned int blocks = gridDim.x * gridDim.y;
+        if (atomicAdd(p2p.done, 1u) == blocks - 1) {
+            atomicExch(p2p.done, 0u);
+            atomicAdd(p2p.seq, 1u);
+        }
+    }
 }
 
 }  // namespace

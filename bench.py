@@ -431,6 +431,13 @@ def run_tp(device, l2, world, rank, T_list=(1, 16, 256, 4096, 8192)):
                 world)
             pt["in_kernel_p2p_us"] = round(p2p, 3)
             pt["p2p_vs_allgather"] = round(p2p / ag, 4)
+            # The same calls replayed from a CUDA graph (no collective library
+            # on this path, so it captures): the device time of a layer call.
+            barrier(world)
+            p2p_g = time_graph_fn_us(
+                lambda i: qkn.qknorm_layerwise_tp_p2p(comm, bufs[i], hq, hk, D, gq, gk, eps),
+                len(bufs))
+            pt["in_kernel_p2p_graph_us"] = round(max_over_ranks(p2p_g, world), 3)
         points.append(pt)
         del bufs, d
         torch.cuda.empty_cache()
@@ -439,7 +446,8 @@ def run_tp(device, l2, world, rank, T_list=(1, 16, 256, 4096, 8192)):
            "workload": "layerwise QK-Norm of 32 query / 8 key heads x 128 split by head over "
                        "%d rank(s), one layer call per step" % world,
            "timing": "eager calls through the Python binding (the exchanges hold NCCL "
-                     "collectives), CUDA events, mean of 50, max over ranks",
+                     "collectives), CUDA events, mean of 50, max over ranks; the in-kernel "
+                     "exchange also from CUDA graphs of 50 calls (median of 5 replays)",
            "points": points}
     if comm is not None:
         torch.cuda.synchronize()

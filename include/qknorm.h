@@ -218,7 +218,10 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
  * lives in that rank's device memory and is mapped into the others with CUDA
  * IPC.  A reader polls its own buffer until every rank's word of the token
  * carries the current call's tag.  Calls alternate between two halves of the
- * buffer, so the buffer is never cleared between calls.
+ * buffer, so the buffer is never cleared between calls.  The call's sequence
+ * number (which picks the half and the tag) is kept in the communicator's
+ * device memory and advanced by each launch, so the calls can be captured in
+ * a CUDA graph and replayed.
  *
  * Waits: the blocks of one token on different ranks wait for one another, so
  * every block of a launch is made resident at once (a cooperative launch;
@@ -247,10 +250,10 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
  *   store into this rank's buffer.
  * qknorm_layerwise_tp_p2p: qkv, gamma_q and gamma_k are host arrays of device
  *   pointers, one entry per rank the communicator serves (1, or world for a
- *   local group, in rank order).  QKN_ERR_TOO_LARGE if T > max_tokens or the
- *   communicator has made 2 * (2^32 - 2) calls; QKN_ERR_UNSUPPORTED if not
- *   connected, the current device is not the communicator's, or the token is
- *   too wide for one block of at most 576 threads with gamma in registers.
+ *   local group, in rank order).  QKN_ERR_TOO_LARGE if T > max_tokens;
+ *   QKN_ERR_UNSUPPORTED if not connected, the current device is not the
+ *   communicator's, or the token is too wide for one block of at most 576
+ *   threads with gamma in registers.
  *   Other arguments and errors as qknorm_layerwise.
  * qknorm_tp_comm_errors: waits of this communicator that gave up, since it was
  *   created (a blocking copy; synchronise with the calls first).

@@ -132,3 +132,47 @@ def test_a_rank_of_its_own_group():
     assert comm.errors() == 0
     assert np.array_equal(gu.stored_bits(x), gu.stored_bits(y))
     comm.close()
+
+
+def test_group_calls_replayed_from_a_cuda_graph():
+    """Two calls captured in one CUDA graph and the graph replayed three times,
+    fresh inputs copied into the buffers before each replay: every replay
+    must match the oracle (inputs and weights are copied into the captured
+    tensors).  Each launch takes a new sequence number (and so
+    a new tag) from device memory; a tag frozen at capture would let a replay
+    take the previous replay's sums for fresh ones."""
+    n, T = 4, 300
+    comm = qkn.TPComm.local(n, max_tokens=T)
+    cases = [synth.make_case(T, 32, 8, 128, seed=700 + i, layerwise=True, scale="lognormal")
+             for i in range(4)]
+    ups = [gu.to_device(_rank_case(cases[0], n, r)[1]) for r in range(n)]
+    xs, gqs, gks = [u[0] for u in ups], [u[1] for u in ups], [u[2] for u in ups]
+    second = [x.clone() for x in xs]  # the second captured call works on its own buffers
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up call outside the capture
+        qkn.qknorm_layerwise_tp_p2p(comm, xs, 8, 2, 128, gqs, gks, 1e-6)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        qkn.qknorm_layerwise_tp_p2p(comm, xs, 8, 2, 128, gqs, gks, 1e-6)
+        qkn.qknorm_layerwise_tp_p2p(comm, second, 8, 2, 128, gqs, gks, 1e-6)
+    for c in cases[1:]:
+        for r, (x, y) in enumerate(zip(xs, second)):
+            fresh, fq, fk = gu.to_device(_rank_case(c, n, r)[1])
+            x.copy_(fresh)
+            y.copy_(fresh)
+            gqs[r].copy_(fq)  # each case draws its own weights
+            gks[r].copy_(fk)
+        g.replay()
+        torch.cuda.synchronize()
+        want = gu.oracle_out(c, "layerwise", c.qkv, c.T)
+        for bufs in (xs, second):
+            out = c.qkv.copy()
+            for r, buf in enumerate(bufs):
+                out[:, _rank_case(c, n, r)[0]] = gu.stored_bits(buf)
+            gu.check(out, want, c.qkv, c.dtype, 40 * 128, "graph replay")
+    assert comm.errors() == 0
+    del g
+    comm.close()
