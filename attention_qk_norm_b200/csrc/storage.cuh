@@ -182,17 +182,10 @@ __device__ __forceinline__ void pdl_wait_then_release()
     asm volatile("griddepcontrol.launch_dependents;");
 }
 
-// cp.async of one 16-byte vector into shared memory through L2 only (.cg),
-// in commit groups.  Each thread waits only for its own groups
-// (cp.async.wait_group), which the hardware completes; there is no spin loop.
-template <int kBytes>
-__device__ __forceinline__ void cp_async(void *smem, const void *gmem)
-{
-    static_assert(kBytes == 16, "vectors are 16 bytes");
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-// The same copy with the destination given as a shared-window address.
+// cp.async of one 16-byte vector into shared memory (destination given as a
+// shared-window address) through L2 only (.cg), in commit groups.  Each
+// thread waits only for its own groups (cp.async.wait_group), which the
+// hardware completes; there is no spin loop.
 __device__ __forceinline__ void cp_async_s(uint32_t smem_addr, const void *gmem)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gmem)

@@ -7,10 +7,11 @@ One step is one call of the hot path over one batch: per-head QK-Norm of the
 head_dim-128, 48-head, T=4096 bf16 workload (the shape of the sglang /
 turbomind kernel table's largest row), in place, through the C ABI.  Steps
 rotate over enough copies of the input that the set is more than four times
-the L2 cache, so every step reads from HBM.  Launches are replayed from CUDA
-graphs of up to 100 steps; the timed region is exactly K steps between a
-barrier plus device synchronisation on both sides, timed with CUDA events
-on the launching stream, max over ranks.
+the L2 cache, so every step reads from HBM.  The K timed steps are replayed
+from CUDA graphs of up to 100 steps, the first opening with the start event
+and the last closing with the end event (event nodes inside the graphs, on
+the launching stream); a barrier plus device synchronisation stands on both
+sides of the timed region, and the time is the max over ranks.
 
 Rank 0 prints one JSON line.  Besides the headline it carries the roofline
 of the kernel, an end-to-end figure through host buffers, the CPU oracle as
