@@ -532,7 +532,7 @@ int launch_tp_vpt(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
     if ((rc = device_info(&dev, &info)) != QKN_OK) return rc;
     if (smem > (size_t)info.smem_optin) return QKN_ERR_UNSUPPORTED;
     if ((rc = resident_blocks(kern, kc, dev, info, threads, smem, &per_sm)) != QKN_OK) return rc;
-    // Every block of every rank served here is resident at once.
+    // At most as many blocks per rank as fit resident at once.
     const int64_t per_rank = (int64_t)info.sms * per_sm / nlocal;
     if (per_rank < 1) return QKN_ERR_UNSUPPORTED;
     const int64_t blocks = T < per_rank ? T : per_rank;
@@ -542,8 +542,18 @@ int launch_tp_vpt(const TPRankPtrs &ptrs, int nlocal, int64_t T, int Hq, int Hk,
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    if (nlocal > 1) {
+        // Several ranks in one launch: their blocks wait on one another, so
+        // the launch is cooperative (all blocks resident, or it fails).
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        // One rank per GPU: a block waits only on blocks of other GPUs'
+        // launches, never on a block of its own launch, so a plain launch
+        // with programmatic dependent launch (as the other kernels) will do.
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ptrs, row_stride, T, Hq, Hk, eps, inv_len_q,

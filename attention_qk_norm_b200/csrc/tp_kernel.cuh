@@ -25,8 +25,10 @@
 // same index on the other ranks to have sent t_{i-1}, which each does in its
 // iteration i-1 before it polls anything of iteration i-1 itself; so by
 // induction over the iterations every poll is eventually satisfied, provided
-// every block of every rank is resident (a cooperative launch) and blocks
-// take the same tokens on every rank.  Each poll still gives up after the
+// every block of every rank gets to run (no more blocks per rank than fit
+// resident; a cooperative launch where one launch serves several ranks, whose
+// blocks then wait on one another) and blocks take the same tokens on every
+// rank.  Each poll still gives up after the
 // communicator's time limit, and the first give-up stops every later wait of
 // the call on this rank.
 #pragma once

@@ -223,10 +223,13 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
  * device memory and advanced by each launch, so the calls can be captured in
  * a CUDA graph and replayed.
  *
- * Waits: the blocks of one token on different ranks wait for one another, so
- * every block of a launch is made resident at once (a cooperative launch;
- * it fails with QKN_ERR_CUDA rather than start partly), and blocks take
- * tokens in the same order on every rank.  Each wait gives up after the
+ * Waits: the blocks of one token on different ranks wait for one another.
+ * Blocks take tokens in the same order on every rank, and a launch never has
+ * more blocks per rank than fit resident at once; a launch that serves
+ * several ranks of a local group, whose blocks wait on one another, is
+ * cooperative (all blocks resident, or it fails with QKN_ERR_CUDA rather than
+ * start partly), while a rank on its own GPU is launched like the other
+ * kernels (its blocks wait only on other GPUs).  Each wait gives up after the
  * communicator's time limit; the first give-up of a call is counted
  * (qknorm_tp_comm_errors, and qknorm_wait_timeouts) and stops every other
  * wait of that call on this rank, so a call whose peer never comes ends
