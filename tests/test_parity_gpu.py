@@ -481,3 +481,45 @@ def test_calls_capture_into_a_cuda_graph():
         assert np.array_equal(gu.stored_bits(x), gu.stored_bits(ex))
         assert np.array_equal(gu.stored_bits(y), gu.stored_bits(ey))
         assert np.array_equal(gu.stored_bits(z), gu.stored_bits(ey))  # one rank: the fused result
+
+
+# ------------------------------------------------------------- random shapes --
+def _random_shapes(n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        dtype = [synth.BF16, synth.FP16, synth.FP32, synth.FP8][int(rng.integers(4))]
+        D = int(rng.choice([64, 128, 256]))
+        ns = int(rng.choice([1, 2, 4, 8]))
+        Hq = int(rng.integers(0, 11)) * ns
+        Hk = int(rng.integers(0 if Hq else 1, 5)) * ns
+        es = {synth.BF16: 2, synth.FP16: 2, synth.FP32: 4, synth.FP8: 1}[dtype]
+        pad = int(rng.integers(0, 4)) * (16 // es)  # keeps rows 16-byte aligned
+        T = int(rng.choice([1, 2, 3, 17, 149, 150, 333, 777]))
+        eps = float(rng.choice([0.0, 1e-6, 1e-5, 1e-2]))
+        out.append(dict(dtype=dtype, D=D, ns=ns, Hq=Hq, Hk=Hk, pad=pad, T=T, eps=eps, seed=seed + i))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _random_shapes(40, 4000), ids=lambda c: "%s-D%d-%dq%dk-n%d-T%d" % (
+    c["dtype"], c["D"], c["Hq"], c["Hk"], c["ns"], c["T"]))
+def test_random_shapes(cfg):
+    """Seeded random shapes through both variants: storage type, head_dim, head
+    counts (multiples of nshards, either kind may be absent), row padding,
+    token counts around the decode / short / long launch-shape boundaries,
+    and eps (0 only where no row is all zero).  Every element against the
+    oracle; layerwise identical for nshards 1 and cfg's nshards."""
+    c = cfg
+    stride = (c["Hq"] + 2 * c["Hk"]) * c["D"] + c["pad"]
+    kw = dict(dtype=c["dtype"], seed=c["seed"], eps=c["eps"], row_stride=stride,
+              scale=None if c["eps"] == 0.0 else "stress")
+    ph = synth.make_case(c["T"], c["Hq"], c["Hk"], c["D"], **kw)
+    full_parity(ph, "per_head", what="random per-head %s" % c)
+    lw = synth.make_case(c["T"], c["Hq"], c["Hk"], c["D"], layerwise=True, **kw)
+    try:
+        a, _ = full_parity(lw, "layerwise", c["ns"], what="random layerwise %s" % c)
+    except qkn.QKNormError as e:  # a token too wide for any launch shape
+        assert e.status == -5, e
+        return
+    b, _ = full_parity(lw, "layerwise", 1, what="random layerwise n=1 %s" % c)
+    assert np.array_equal(a, b), "layerwise output depends on nshards"

@@ -30,9 +30,9 @@ def _rank_case(c, n, r):
     k = c.Hq * D + np.arange(r * hk * D, (r + 1) * hk * D)
     v = (c.Hq + c.Hk) * D + np.arange(r * hk * D, (r + 1) * hk * D)
     cols = np.concatenate([q, k, v])
+    gk = None if c.gamma_k is None else c.gamma_k[r * hk * D:(r + 1) * hk * D]
     sub = synth.Case(np.ascontiguousarray(c.qkv[:, cols]), c.gamma_q[r * hq * D:(r + 1) * hq * D],
-                     c.gamma_k[r * hk * D:(r + 1) * hk * D], c.T, hq, hk, D, (hq + 2 * hk) * D,
-                     c.dtype, c.eps, True)
+                     gk, c.T, hq, hk, D, (hq + 2 * hk) * D, c.dtype, c.eps, True)
     return cols, sub
 
 
@@ -176,3 +176,32 @@ def test_group_calls_replayed_from_a_cuda_graph():
     assert comm.errors() == 0
     del g
     comm.close()
+
+
+def _random_groups(n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        dtype = [synth.BF16, synth.FP16, synth.FP32, synth.FP8][int(rng.integers(4))]
+        D = int(rng.choice([64, 128, 256]))
+        world = int(rng.choice([2, 4, 8]))
+        hq = int(rng.integers(0, 5))
+        hk = int(rng.integers(0 if hq else 1, 3))
+        T = int(rng.choice([1, 5, 149, 333]))
+        out.append(dict(dtype=dtype, D=D, world=world, Hq=hq * world, Hk=hk * world, T=T,
+                        seed=seed + i))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _random_groups(16, 6000), ids=lambda c: "%s-D%d-%dq%dk-w%d-T%d" % (
+    c["dtype"], c["D"], c["Hq"], c["Hk"], c["world"], c["T"]))
+def test_random_groups(cfg):
+    """Seeded random groups of the in-kernel exchange: storage type, head_dim,
+    group size, heads per rank (either kind may be absent) and T; every
+    element against the oracle of the whole vectors."""
+    c = synth.make_case(cfg["T"], cfg["Hq"], cfg["Hk"], cfg["D"], dtype=cfg["dtype"],
+                        seed=cfg["seed"], layerwise=True, scale="stress", zero_frac=0.02,
+                        outlier_frac=0.02)
+    out = run_group(c, cfg["world"])
+    want = gu.oracle_out(c, "layerwise", c.qkv, c.T)
+    gu.check(out, want, c.qkv, c.dtype, (c.Hq + c.Hk) * c.D, "random group %s" % cfg)
