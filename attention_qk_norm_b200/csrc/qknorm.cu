@@ -195,7 +195,7 @@ template <typename TS, int D, bool kHasK, bool kSplit = false>
 int launch_per_head_k(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, const float *gq,
                       const float *gk, float eps, cudaStream_t stream)
 {
-    constexpr int U = kPerHeadRowsInFlight;
+    constexpr int U = per_head_rows_in_flight<TS>();
     constexpr int kNV = D / Storage<TS>::kVec;
     constexpr int kLPR = kNV < 32 ? kNV : 32;
     auto kern = qkn_per_head_kernel<TS, D, U, kHasK, kSplit>;
