@@ -12,10 +12,6 @@
 namespace {
 
 // --------------------------------------------------------------- layerwise --
-// Stages of the staging ring (one token staged ahead of the one being worked
-// on).  Three stages measured 2-11% slower for bf16/fp16/fp32 on B200 (a
-// resident block fewer) and no better for FP8.
-constexpr int kLayerwiseStages = 2;
 
 // How warp_sumsq reduces the nh head partials of one vector (q or k).  The
 // host fills it once per launch, so the token loop divides nothing.
@@ -23,10 +19,13 @@ constexpr int kLayerwiseStages = 2;
 //              of two dividing nh (0 when nh == 0);
 //   per_lane:  heads each of those lanes sums, in order (nh / used);
 //   per_shard: lanes per emulated shard (used / nshards).
+//   warps:     with the warp tree (below), the warps whose sums make up
+//              the vector (0 for both vectors when it is not used).
 struct SumPlan {
     int used;
     int per_lane;
     int per_shard;
+    int warps;
 };
 
 // Sum of squares of one vector from its head partials part[0..nh), computed
@@ -55,6 +54,25 @@ __device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p,
     for (int o = 1; o < 32; o <<= 1)
         if (o < p.used) v += __shfl_xor_sync(0xffffffffu, v, o);
     return __shfl_sync(0xffffffffu, v, 0);
+}
+
+// The warp tree.  When a vector's head count nh is a power of two up to 64,
+// warp_sumsq's tree is the balanced binary tree over head index (with 64
+// heads each lane first adds two neighbours, which is the tree's lowest
+// level).  A block of a plain launch whose warps each hold hpw = 32 / LPH
+// whole heads of one vector, hpw dividing Hq, then holds that tree's
+// subtrees warp by warp: each warp forms its subtree with xor butterflies
+// at lane distances LPH, 2 LPH, ... 16 (head distances 1, 2, ...,
+// hpw / 2) before the block barrier, and after it every lane adds the
+// vector's n <= 8 warp sums in the tree's remaining levels.  The association
+// is the same, so the bits are too; lanes past the last head add zeros,
+// which leaves a sum of squares unchanged.
+__device__ __forceinline__ float warp_tree_sum(const float *w, int n)
+{
+    if (n == 1) return w[0];
+    if (n == 2) return w[0] + w[1];
+    if (n == 4) return (w[0] + w[1]) + (w[2] + w[3]);
+    return ((w[0] + w[1]) + (w[2] + w[3])) + ((w[4] + w[5]) + (w[6] + w[7]));
 }
 
 // ---- cluster exchange of head partials (transaction barriers) --
@@ -124,12 +142,27 @@ enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 //                  staged.
 enum LayerwiseSchedule { kSchedRing = 0, kSchedOverlap = 1, kSchedDirect = 2 };
 
+// Stages of the staging ring: two (one token staged ahead of the one being
+// worked on), three for FP8 on the overlap schedule.  Measured on B200: a
+// third stage costs bf16/fp16/fp32 2-11% (a resident block fewer, or, for
+// fp32 on the overlap schedule, 2-9% with the same blocks), while FP8, whose
+// tokens are short and whose four resident blocks keep only 20 KB per SM in
+// flight with two stages, gains 4-5% (32q/8kv, T = 8192 to 32768); a fourth
+// stage is slower again.
+template <typename TS, int kSched>
+__host__ __device__ constexpr int layerwise_stages()
+{
+    return kSched == kSchedDirect                                  ? 0
+           : (kSched == kSchedOverlap && Storage<TS>::kVec == 16) ? 3
+                                                                  : 2;
+}
+
 // A token's heads are split over the CL blocks of a thread-block cluster
 // (CL = 1 for a plain launch): block c of a cluster owns heads
 // [c*hc, (c+1)*hc), hc = heads/CL, with roundup32(hc * NV / VPT) threads;
 // thread (h, l) owns vectors l, l + LPH, ... of head h (LPH = NV / VPT lanes
 // per head), and thread l == 0 is the head's owner.  Dynamic shared memory
-// per block: the ring's kLayerwiseStages stages of this block's part of a
+// per block: the ring's layerwise_stages() stages of this block's part of a
 // token (hc*D*sizeof(TS) bytes each; none with the direct schedule), two
 // buffers of `heads` fp32 head partials (alternating per token), then the
 // two exchange barriers (CL > 1).  With
@@ -158,7 +191,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     // register caps leave no room for pair alignment, multiply in scalars
     // (the same bits either way).
     constexpr bool kPacked = kOverlap;
-    constexpr int NST = kDirect ? 0 : kLayerwiseStages;  // stages of the ring
+    constexpr int NST = layerwise_stages<TS, kSched>();  // stages of the ring
     constexpr bool kExchange = kCluster && kMode != kApply;
     // Vector loops unroll fully when gamma sits in registers (indexed by v);
     // with gamma in L1 the long loops unroll by 8.
@@ -328,6 +361,11 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 // thread sends its next partial, which any sender of that phase
                 // has to wait for.
                 if (threadIdx.x == 0 && !timed_out) mbar_arm(&bar[pb], token_bytes);
+            } else if (plan_q.warps | plan_k.warps) {
+#pragma unroll
+                for (int o = kLPH; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0) pp[threadIdx.x / 32] = s;
+                __syncthreads();
             } else {
                 if (active && l == 0) pp[h] = s;
                 __syncthreads();
@@ -342,6 +380,10 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                         aux[2 * t + 1] = sk;
                     }
                 }
+            } else if (!kExchange && (plan_q.warps | plan_k.warps)) {
+                if (need_q) rq = rsqrtf(warp_tree_sum(pp, plan_q.warps) * inv_len_q + eps);
+                if (need_k)
+                    rk = rsqrtf(warp_tree_sum(pp + plan_q.warps, plan_k.warps) * inv_len_k + eps);
             } else {
                 if (need_q) rq = rsqrtf(warp_sumsq(pp, plan_q, lane) * inv_len_q + eps);
                 if (need_k) rk = rsqrtf(warp_sumsq(pp + Hq, plan_k, lane) * inv_len_k + eps);

@@ -260,6 +260,39 @@ def test_layerwise_decode_sizes(T, Hq, Hk, D, dtype):
     assert np.array_equal(gu.stored_bits(x), outs[0])
 
 
+@pytest.mark.parametrize("dtype,T,Hq,Hk,D,ns", [
+    (synth.FP8, 4000, 64, 8, 128, (1, 8)),   # overlap; 8 query warps, 64-head tree
+    (synth.FP8, 3000, 8, 4, 128, (1, 4)),    # key warp padded past its 4 heads
+    (synth.FP8, 500, 0, 16, 128, (1, 8)),    # key heads only
+    (synth.FP8, 500, 16, 0, 64, (1, 8)),     # query heads only, 16 heads per warp
+    (synth.FP8, 2000, 32, 8, 256, (1, 8)),   # 4 heads per warp
+    (synth.FP8, 300, 4, 4, 128, (1, 4)),     # a warp holds both kinds: head partials
+    (synth.FP8, 300, 12, 4, 128, (1, 4)),    # 12 is no power of two: head partials
+    (synth.FP8, 300, 128, 8, 128, (1, 8)),   # 16 query warps: head partials
+    (synth.BF16, 64, 32, 8, 128, (1, 8)),    # decode size, direct schedule
+    (synth.BF16, 1000, 32, 8, 128, (1, 8)),  # short input, twice the vectors per thread
+    (synth.BF16, 1000, 16, 16, 64, (1, 8)),
+    (synth.FP32, 500, 32, 8, 128, (1, 8)),
+])
+def test_layerwise_warp_tree(dtype, T, Hq, Hk, D, ns):
+    """Shapes on both sides of the warp tree's conditions (FP8 launches and
+    short inputs; each vector a power of two of heads up to 64, whole warps
+    per vector, at most 8 warps per vector).  Every element against the
+    oracle, the same bits for every nshards, and the same bits as the two
+    tensor-parallel steps, whose partials step always sums head partials
+    in warp_sumsq's order at the same vectors per thread."""
+    c = synth.make_case(T, Hq, Hk, D, dtype=dtype, seed=400 + T + Hq + D, layerwise=True,
+                        scale="stress", zero_frac=0.02, outlier_frac=0.02)
+    outs = [full_parity(c, "layerwise", n, what="warp tree %s %d/%d n=%d" % (dtype, Hq, Hk, n))[0]
+            for n in ns]
+    assert np.array_equal(outs[0], outs[1])
+    x, gq, gk = gu.to_device(c)
+    sums = qkn.qknorm_layerwise_partials(x, Hq, Hk, D)
+    qkn.qknorm_layerwise_apply(x, Hq, Hk, D, gq, gk, sums, Hq * D, Hk * D, c.eps)
+    torch.cuda.synchronize()
+    assert np.array_equal(gu.stored_bits(x), outs[0])
+
+
 @pytest.mark.parametrize("dtype", (synth.BF16, synth.FP8))
 def test_layerwise_gamma_through_l1(dtype):
     """129 heads of 256 (odd, so no cluster split): gamma cannot stay in
