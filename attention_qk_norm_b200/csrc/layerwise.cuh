@@ -59,14 +59,14 @@ __device__ __forceinline__ float warp_sumsq(const float *part, const SumPlan &p,
 // The warp tree.  When a vector's head count nh is a power of two up to 64,
 // warp_sumsq's tree is the balanced binary tree over head index (with 64
 // heads each lane first adds two neighbours, which is the tree's lowest
-// level).  A block of a plain launch whose warps each hold hpw = 32 / LPH
-// whole heads of one vector, hpw dividing Hq, then holds that tree's
-// subtrees warp by warp: each warp forms its subtree with xor butterflies
-// at lane distances LPH, 2 LPH, ... 16 (head distances 1, 2, ...,
-// hpw / 2) before the block barrier, and after it every lane adds the
-// vector's n <= 8 warp sums in the tree's remaining levels.  The association
-// is the same, so the bits are too; lanes past the last head add zeros,
-// which leaves a sum of squares unchanged.
+// level).  A block of a plain launch with gamma in registers, whose warps
+// each hold hpw = 32 / LPH whole heads of one vector (hpw dividing Hq),
+// then holds that tree's subtrees warp by warp: each warp forms its subtree
+// with xor butterflies at lane distances LPH, 2 LPH, ... 16 (head distances
+// 1, 2, ..., hpw / 2) before the block barrier, and after it every lane adds
+// the vector's n <= 8 warp sums in the tree's remaining levels.  The
+// association is the same, so the bits are too; lanes past the last head add
+// zeros, which leaves a sum of squares unchanged.
 __device__ __forceinline__ float warp_tree_sum(const float *w, int n)
 {
     if (n == 1) return w[0];
@@ -224,6 +224,22 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
     const bool need_k = Hk > 0 && warp_last_head >= Hq;
     const int64_t first = blockIdx.x / cl, stride = gridDim.x / cl;  // this cluster's tokens
 
+    // This thread's vectors of the first tokens (those the ring stages first,
+    // or the one the direct schedule loads) into L2 before the wait.  Not in
+    // the apply step, which follows the all-reduce (a grid that lets no
+    // dependent start early), nor with gamma read through L1.
+    if constexpr (kGammaRegs && kMode != kApply) {
+        if (active) {
+            const TS *row = qkv + first * row_stride + (int64_t)h * D + l * kVec;
+#pragma unroll
+            for (int i = 0; i < (NST > 1 ? NST - 1 : 1); ++i)
+                if (first + i * stride < T) {
+#pragma unroll
+                    for (int v = 0; v < VPT; ++v)
+                        prefetch_l2(row + i * stride * row_stride + v * kLPH * kVec);
+                }
+        }
+    }
     pdl_wait_then_release();
     // This thread's head weights (the partials step has none).
     const float *gb = gamma_q;
@@ -361,7 +377,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                 // thread sends its next partial, which any sender of that phase
                 // has to wait for.
                 if (threadIdx.x == 0 && !timed_out) mbar_arm(&bar[pb], token_bytes);
-            } else if (plan_q.warps | plan_k.warps) {
+            } else if (kGammaRegs && (plan_q.warps | plan_k.warps)) {
 #pragma unroll
                 for (int o = kLPH; o < 32; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
                 if (lane == 0) pp[threadIdx.x / 32] = s;
@@ -380,7 +396,7 @@ layerwise_tokens(TS *__restrict__ qkv, int64_t row_stride, int64_t T, int Hq, in
                         aux[2 * t + 1] = sk;
                     }
                 }
-            } else if (!kExchange && (plan_q.warps | plan_k.warps)) {
+            } else if (kGammaRegs && !kExchange && (plan_q.warps | plan_k.warps)) {
                 if (need_q) rq = rsqrtf(warp_tree_sum(pp, plan_q.warps) * inv_len_q + eps);
                 if (need_k)
                     rk = rsqrtf(warp_tree_sum(pp + plan_q.warps, plan_k.warps) * inv_len_k + eps);

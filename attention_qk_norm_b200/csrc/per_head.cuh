@@ -65,7 +65,6 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
     // scalars.
     constexpr bool kPacked = kVec == 16;
 
-    pdl_wait_then_release();
     uint64_t block = blockIdx.x, nblocks = gridDim.x;
     if constexpr (kSplit) {
         if (blockIdx.x >= q_blocks) {  // key rows: the columns after the Hq query heads
@@ -84,23 +83,8 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
     const uint64_t group = tid / kLPR;
     const uint64_t ngroups = (nblocks * blockDim.x) / kLPR;
 
-    // This lane's columns are fixed: vectors lane, lane + LPR, ... of a row.
-    float gq[kEPL], gk[kHasK ? kEPL : 1];
-#pragma unroll
-    for (int v = 0; v < kVPL; ++v) {
-        const int col = (lane + v * kLPR) * kVec;
-        float tq[kVec];
-        load_gamma<kVec>(gamma_q + col, tq);
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) gq[v * kVec + e] = tq[e];
-        if constexpr (kHasK) {
-            float tk[kVec];
-            load_gamma<kVec>(gamma_k + col, tk);
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) gk[v * kVec + e] = tk[e];
-        }
-    }
-
+    // The first rows' (token, head) pairs depend on the arguments only: they
+    // are found, and the rows' lines prefetched into L2, before the wait.
     // The first rows and the step are below U * ngroups (at most a few
     // hundred thousand), so 32-bit division can find their (token, head)
     // pairs; it shortens the start of the single-weight kernel (measured
@@ -132,6 +116,32 @@ qkn_per_head_kernel(TS *__restrict__ qkv, int64_t row_stride, int64_t T, uint32_
         dt = (int64_t)(step / heads);
         dh = (uint32_t)(step - (uint64_t)dt * heads);
     }
+#pragma unroll
+    for (int k = 0; k < U; ++k)
+        if (t[k] < T) {
+            const V *p = reinterpret_cast<const V *>(qkv + t[k] * row_stride + (int64_t)h[k] * D);
+#pragma unroll
+            for (int v = 0; v < kVPL; ++v) prefetch_l2(p + lane + v * kLPR);
+        }
+    pdl_wait_then_release();
+
+    // This lane's columns are fixed: vectors lane, lane + LPR, ... of a row.
+    float gq[kEPL], gk[kHasK ? kEPL : 1];
+#pragma unroll
+    for (int v = 0; v < kVPL; ++v) {
+        const int col = (lane + v * kLPR) * kVec;
+        float tq[kVec];
+        load_gamma<kVec>(gamma_q + col, tq);
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) gq[v * kVec + e] = tq[e];
+        if constexpr (kHasK) {
+            float tk[kVec];
+            load_gamma<kVec>(gamma_k + col, tk);
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) gk[v * kVec + e] = tk[e];
+        }
+    }
+
     const uint64_t rows = (uint64_t)T * heads;
     // The trip count is the same for every thread, so whole warps reach each
     // shuffle together; rows past the end contribute zeros and store nothing.

@@ -26,9 +26,12 @@
 // thread scales its vectors by the inverse RMS of its vector.
 //
 // Both kernels are launched with programmatic dependent launch: they wait on
-// griddepcontrol.wait before their first global memory access, so a kernel
-// earlier in the stream always finishes first, and they allow the next
-// kernel to be scheduled as soon as all of their blocks are resident.  The
+// griddepcontrol.wait before their first load or store, so a kernel earlier
+// in the stream always finishes first, and they allow the next kernel to be
+// scheduled as soon as all of their blocks are resident.  Before the wait a
+// block only computes its first rows' addresses and prefetches those rows
+// into L2 (prefetch_l2), which overlaps the latency of its first loads with
+// the draining of the grid before it.  The
 // only wait between blocks is inside a thread-block cluster of the layerwise
 // kernel, whose blocks the hardware schedules together; each such wait gives
 // up after a time limit, so no kernel here can hang.
@@ -492,7 +495,7 @@ int launch_layerwise(void *qkv, int64_t T, int Hq, int Hk, int64_t row_stride, c
     // and 1-2% on short bf16 inputs (T = 256 to 4096), where the chain after
     // the barrier is a larger part of a token's time; on long bf16 / fp16
     // inputs the per-head partials measured 1% faster.
-    if (kMode == kFused && cluster == 1 && (kVec == 16 || short_launch))
+    if (kMode == kFused && cluster == 1 && chosen * kVec <= 32 && (kVec == 16 || short_launch))
         set_warp_tree(plan_q, plan_k, Hq, Hk, 32 / (kNV / chosen));
 #define QKN_LW_CASE(V)                                                                         \
     case V:                                                                                    \

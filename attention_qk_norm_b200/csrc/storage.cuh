@@ -182,6 +182,18 @@ __device__ __forceinline__ void pdl_wait_then_release()
     asm volatile("griddepcontrol.launch_dependents;");
 }
 
+// An L2 prefetch hint for the line holding p (an address inside a buffer the
+// kernel reads).  A block that starts while the grid before it is still
+// draining issues these for its first rows before griddepcontrol.wait, so
+// that its first loads after the wait find their lines in L2.  A prefetch
+// returns no data to the thread, and every SM's accesses to a line meet in
+// the L2, which the hardware keeps coherent, so a load after the wait still
+// sees every write of the preceding grid.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // cp.async of one 16-byte vector into shared memory (destination given as a
 // shared-window address) through L2 only (.cg), in commit groups.  Each
 // thread waits only for its own groups (cp.async.wait_group), which the

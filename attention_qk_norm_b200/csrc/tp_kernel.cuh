@@ -134,6 +134,13 @@ qkn_layerwise_tp_kernel(TPRankPtrs ptrs, int64_t row_stride, int64_t T, int Hq, 
     const int world = p2p.world;
     const int64_t first = blockIdx.x, stride = gridDim.x;
 
+    // This thread's vectors of its first token into L2 before the wait (a
+    // hint that returns no data; see prefetch_l2).
+    if (active && first < T) {
+        const TS *row = qkv + first * row_stride + (int64_t)hl * D + l * kVec;
+#pragma unroll
+        for (int v = 0; v < VPT; ++v) prefetch_l2(row + v * kLPH * kVec);
+    }
     pdl_wait_then_release();
     // This call's buffer half and tag (tp_exchange.h), from the sequence
     // number that the previous launch left behind.
