@@ -36,17 +36,50 @@ def nvcc() -> str:
     return found
 
 
-def kernel_source_sha256() -> str:
-    """SHA-256 over the library's CUDA sources (file names and contents, in
-    name order); recorded ncu counters are valid only for the sources they
-    were taken from."""
+def code_only(text: str) -> str:
+    """C/C++/CUDA source text without its comments and with each run of
+    whitespace made one space: what the compiler reads."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":  # a string or character literal, copied whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_sources() -> list:
+    """The files compiled into the kernels: the translation unit and the
+    headers beside it."""
+    return sorted(SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                             if f.endswith((".cuh", ".h"))])
+
+
+def kernel_source_sha256(read=None) -> str:
+    """SHA-256 over the code of the library's CUDA sources (file names and
+    their text without comments, in name order); recorded ncu counters are
+    valid only for the code they were taken from.  ``read(path)`` returns a
+    file's text (default: the file on disk)."""
     import hashlib
 
+    read = read or (lambda p: open(p, encoding="utf-8").read())
     h = hashlib.sha256()
-    for p in sorted(SOURCES + HEADERS[1:]):
+    for p in kernel_sources():
         h.update(os.path.basename(p).encode() + b"\0")
-        with open(p, "rb") as f:
-            h.update(f.read())
+        h.update(code_only(read(p)).encode())
     return h.hexdigest()
 
 

@@ -130,9 +130,9 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 enum LayerwiseMode { kFused = 0, kPartials = 1, kApply = 2 };
 
 // How a launch moves each token through its block.
-//   kSchedRing:    a two-stage cp.async ring in shared memory (the next token
-//                  is fetched while this one is processed), then a second pass
-//                  over the staged token to scale it.
+//   kSchedRing:    a cp.async ring in shared memory (the next token is
+//                  fetched while this one is processed; layerwise_stages),
+//                  then a second pass over the staged token to scale it.
 //   kSchedOverlap: the ring, with x * gamma formed in the first pass, while
 //                  the token's partials are still being combined (SwiftQK's
 //                  overlap), and kept in registers: no second pass.

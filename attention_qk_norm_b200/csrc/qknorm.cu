@@ -16,9 +16,10 @@
 //
 // Layerwise (SwiftQK abstract; review key_machinery): a persistent block
 // (or thread-block cluster, for tokens too wide for one block) walks tokens
-// with a grid stride.  Each thread copies its vectors of the next token into
-// a two-stage shared-memory ring with cp.async while it works on the current
-// one (at decode sizes it loads them straight into registers instead).  The
+// with a grid stride.  Each thread copies its vectors of the next token (the
+// next two for FP8 on long inputs) into a shared-memory ring with cp.async
+// while it works on the current one (at decode sizes it loads them straight
+// into registers instead).  The
 // per-head partial sums of squares meet in shared memory behind one barrier
 // (across a cluster, on transaction barriers); then each warp, for the
 // vectors (q, k) its threads hold, forms every emulated shard's fp32 partial

@@ -111,8 +111,9 @@ int qknorm_per_head(void *qkv, int dtype, int64_t T, int Hq, int Hk, int D, int6
  * The reduction is a fixed tree whose subtrees are the shards, so the output
  * is bit-identical for every valid nshards.  A token's heads are split over
  * a thread-block cluster of 1, 2, 4 or 8 blocks (C, which must divide
- * Hq + Hk); each block keeps two tokens' worth of its heads staged in shared
- * memory, so 2 * (Hq + Hk) / C * D * sizeof(element) + 8 * (Hq + Hk) + 16
+ * Hq + Hk); each block keeps S = 2 tokens' worth of its heads staged in
+ * shared memory (S = 3 for FP8 on inputs long enough for the x * gamma
+ * overlap), so S * (Hq + Hk) / C * D * sizeof(element) + 8 * (Hq + Hk) + 16
  * bytes must fit the device's opt-in shared memory per block (227 KiB on
  * B200) for the cluster size chosen, else QKN_ERR_UNSUPPORTED.  The blocks of
  * a cluster pass head partials to one another through distributed shared
