@@ -5,8 +5,8 @@
 // every element is scaled by 1/sqrt(S_global/H + eps)).
 //
 // Each rank owns a receive buffer in its own device memory, which the other
-// ranks of the group write through CUDA IPC mappings (plain peer stores over
-// NVLink; no multicast).  For every token a rank stores its two fp32 partial
+// ranks of the group write through CUDA IPC mappings (plain point-to-point
+// peer stores over NVLink, one destination each).  For every token a rank stores its two fp32 partial
 // sums of squares (its q heads, its k heads) into its slot of every rank's
 // buffer, itself included, each as ONE 64-bit word {fp32 value, 32-bit call
 // tag}: value and flag travel in a single naturally aligned store, so a

@@ -214,8 +214,9 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
  * gamma_q / gamma_k are this rank's slices (Hq*D and Hk*D floats).
  *
  * The exchange: each of a rank's partial sums travels as one 8-byte word
- * {fp32 value, 32-bit call tag}, written with a single peer store (no
- * multicast, no collective library) into the receive buffer of each rank, which
+ * {fp32 value, 32-bit call tag}, written with a single point-to-point peer
+ * store (one destination per store, no collective library) into the receive
+ * buffer of each rank, which
  * lives in that rank's device memory and is mapped into the others with CUDA
  * IPC.  A reader polls its own buffer until every rank's word of the token
  * carries the current call's tag.  Calls alternate between two halves of the
