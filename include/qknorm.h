@@ -216,9 +216,8 @@ int qknorm_layerwise_noalloc(void *qkv, int dtype, int64_t T, int Hq, int Hk, in
  * The exchange: each of a rank's partial sums travels as one 8-byte word
  * {fp32 value, 32-bit call tag}, written with a single point-to-point peer
  * store (one destination per store, no collective library) into the receive
- * buffer of each rank, which
- * lives in that rank's device memory and is mapped into the others with CUDA
- * IPC.  A reader polls its own buffer until every rank's word of the token
+ * buffer of each rank, which lives in that rank's device memory and is
+ * mapped into the others with CUDA IPC.  A reader polls its own buffer until every rank's word of the token
  * carries the current call's tag.  Calls alternate between two halves of the
  * buffer, so the buffer is never cleared between calls.  The call's sequence
  * number (which picks the half and the tag) is kept in the communicator's
