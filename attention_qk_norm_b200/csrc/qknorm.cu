@@ -607,7 +607,8 @@ struct LayerwiseTP {
         const int threads = (heads * (kNV / vpt) + 31) / 32 * 32;
         const float inv_len_q = Hq > 0 ? 1.0f / len_q : 0.f;
         const float inv_len_k = Hk > 0 ? 1.0f / len_k : 0.f;
-        const SumPlan plan_q = sum_plan(Hq, 1), plan_k = sum_plan(Hk, 1);
+        SumPlan plan_q = sum_plan(Hq, 1), plan_k = sum_plan(Hk, 1);
+        set_warp_tree(plan_q, plan_k, Hq, Hk, 32 / (kNV / vpt));
 #define QKN_TP_CASE(V)                                                                         \
     case V:                                                                                    \
         if constexpr (layerwise_vpt_ok<TS, D, V>() && layerwise_gamma_regs<TS, V>())           \

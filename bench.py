@@ -807,6 +807,10 @@ PROFILE_CASES = {
     # GPU (one cooperative launch serves all ranks).
     "tp_group": dict(kind="tp_group", T=4096, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
                      nshards=8, seed=1007),
+    # One rank holding every head: the exchange kernel as a rank on its own
+    # GPU launches it (programmatic dependent launch, not cooperative).
+    "tp_rank": dict(kind="tp_group", T=8192, Hq=32, Hk=8, D=128, dtype="bf16", eps=1e-6,
+                    nshards=1, seed=1008),
     # 128 heads of 256: too wide for one block, so 2-block clusters exchange
     # head partials through distributed shared memory.
     "layerwise_cluster": dict(kind="layerwise", T=4096, Hq=112, Hk=16, D=256, dtype="bf16",
